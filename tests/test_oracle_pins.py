@@ -1,0 +1,370 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself.
+
+Brute force on tiny inputs, closed forms, invariants of exact softmax attention,
+library rounding routines and the OCP FP8 E4M3 value table.  A plausible slip in
+the oracle (a dropped rescale, a wrong block index, a transposed operand, a
+wrong rounding mode) fails at least one of these.
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from quantized_attention_06_b200.inputs import WORKLOADS, generate
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- rounding
+
+def test_round_binary_matches_numpy_fp16():
+    rng = np.random.default_rng(11)
+    x = np.concatenate([
+        rng.standard_normal(200000) * 10.0 ** rng.uniform(-9, 4.5, 200000),
+        np.array([2.0 ** -24 * 0.5, 2.0 ** -24 * 1.5, 2.0 ** -14, 65504.0, 1.0 + 2.0 ** -11]),
+    ])
+    x = x[np.abs(x) < 65504.0]
+    mine = orc.round_binary(x, p=11, emin=-14)
+    lib = x.astype(np.float16).astype(np.float64)
+    assert np.array_equal(mine, lib)
+
+
+def test_round_binary_matches_torch_bf16():
+    rng = np.random.default_rng(12)
+    x = (rng.standard_normal(200000) * 10.0 ** rng.uniform(-30, 30, 200000)).astype(np.float32)
+    mine = orc.round_binary(x.astype(np.float64), p=8, emin=-126)
+    lib = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(mine, lib)
+
+
+def _ocp_points():
+    pts = []
+    with open(os.path.join(GOLDEN, "e4m3_ocp_points.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            code, val = line.split()
+            pts.append((int(code, 16), float(val)))
+    return pts
+
+
+def test_e4m3_decode_matches_ocp_table():
+    for code, val in _ocp_points():
+        got = orc.e4m3_decode(np.array([code]))[0]
+        if math.isnan(val):
+            assert math.isnan(got)
+        else:
+            assert got == val and math.copysign(1, got) == math.copysign(1, val), hex(code)
+
+
+def test_e4m3_all_codes_round_trip_and_monotone():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F])
+    vals = orc.e4m3_decode(codes)
+    assert np.array_equal(orc.e4m3_round(vals), vals)
+    assert np.array_equal(orc.e4m3_encode(vals), codes.astype(np.uint8))
+    pos = orc.e4m3_decode(np.arange(0, 0x7F))
+    assert np.all(np.diff(pos) > 0)
+    assert pos[-1] == 448.0 and pos[1] == 2.0 ** -9
+
+
+def test_e4m3_midpoints_tie_to_even_and_saturate():
+    pos = orc.e4m3_decode(np.arange(0, 0x7F))
+    lo, hi = pos[:-1], pos[1:]
+    mid = (lo + hi) / 2
+    r = orc.e4m3_round(mid)
+    even = np.where(np.arange(0, 0x7E) % 2 == 0, lo, hi)   # even code = even mantissa
+    assert np.array_equal(r, even)
+    assert np.array_equal(orc.e4m3_round(np.nextafter(mid, np.inf)), hi)
+    assert np.array_equal(orc.e4m3_round(np.nextafter(mid, -np.inf)), lo)
+    assert np.array_equal(orc.e4m3_round(-mid), -even)
+    assert list(orc.e4m3_round(np.array([460.0, 480.0, 1e9, -1e9]))) == [448.0, 448.0, 448.0, -448.0]
+
+
+def test_e4m3_round_matches_torch_float8():
+    rng = np.random.default_rng(13)
+    x = (rng.standard_normal(300000) * 10.0 ** rng.uniform(-4, 2.6, 300000)).astype(np.float32)
+    x = x[np.abs(x) <= 448.0]
+    lib = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(orc.e4m3_round(x.astype(np.float64)), lib)
+
+
+# ---------------------------------------------------------------- quantizers
+
+def test_k_mean_closed_form():
+    rng = np.random.default_rng(1)
+    d, n = 16, 300
+    base = rng.integers(-50, 50, size=(n, d)).astype(np.float32)
+    base -= base.mean(axis=0, keepdims=True).round()          # integer data
+    mu_exact = base.astype(np.float64).sum(axis=0) / n
+    assert np.array_equal(orc.k_channel_mean(base), mu_exact.astype(np.float32))
+    # a per-channel constant shift moves the mean by exactly that constant
+    c = np.arange(d, dtype=np.float32) * 0.25
+    assert np.array_equal(orc.k_channel_mean(base + c) - orc.k_channel_mean(base), c)
+
+
+def test_int8_quantization_is_lossless_on_grid_values():
+    rng = np.random.default_rng(2)
+    for blk in (orc.BLKQ, orc.BLKK):
+        n, d = 3 * blk - 17, 64                                  # ragged last block
+        ints = rng.integers(-126, 127, size=(n, d))
+        for b in range(0, n, blk):
+            ints[b, 0] = 127 if b % 2 else -127                   # one +-127 per block
+        cs = np.float32([0.5, 0.25, 2.0])
+        x = np.concatenate([ints[b:b + blk] * cs[i] for i, b in enumerate(range(0, n, blk))])
+        codes, scales = orc.quantize_int8_blocks(x.astype(np.float32), blk)
+        assert codes.shape == (3 * blk, d)
+        assert np.array_equal(codes[:n], ints.astype(np.int8))
+        assert np.all(codes[n:] == 0)
+        assert np.array_equal(scales, cs)
+
+
+def test_int8_quantization_error_bound_and_block_partition():
+    rng = np.random.default_rng(3)
+    n, d = 5 * orc.BLKK + 9, 32
+    # each token block has its own magnitude: a scale taken from the wrong
+    # block (or reduced over channels instead of tokens) breaks the bound
+    mag = np.repeat(2.0 ** np.arange(6), orc.BLKK)[:n]
+    x = (rng.standard_normal((n, d)) * mag[:, None]).astype(np.float32)
+    codes, scales = orc.quantize_int8_blocks(x, orc.BLKK)
+    for b in range(6):
+        rows = slice(b * orc.BLKK, min(n, (b + 1) * orc.BLKK))
+        a = np.abs(x[rows]).max()
+        assert scales[b] == np.float32(a / np.float32(127))
+        err = np.abs(codes[rows].astype(np.float64) * scales[b] - x[rows])
+        assert np.all(err <= 0.5 * scales[b] * (1 + 1e-5))
+        assert np.abs(codes[rows]).max() == 127
+
+
+def test_int8_zero_block():
+    x = np.zeros((orc.BLKQ + 5, 8), dtype=np.float32)
+    x[orc.BLKQ:] = 1.0
+    codes, scales = orc.quantize_int8_blocks(x, orc.BLKQ)
+    assert scales[0] == 0 and np.all(codes[:orc.BLKQ] == 0)
+    assert scales[1] == np.float32(1 / np.float32(127)) and np.all(codes[orc.BLKQ:orc.BLKQ + 5] == 127)
+
+
+def test_v_e4m3_quantization_bound():
+    rng = np.random.default_rng(4)
+    v = (rng.standard_normal((333, 24)) * np.exp2(rng.integers(-6, 6, 24))[None, :]).astype(np.float32)
+    v[:, 3] = 0.0                                                # an all-zero channel
+    codes, sv = orc.quantize_v_e4m3(v)
+    deq = orc.e4m3_decode(codes) * sv.astype(np.float64)[None, :]
+    # e4m3 keeps 3 mantissa bits: half-ulp <= 2^-4 relative, 2^-10 * sv absolute below 2^-6
+    bound = np.maximum(2.0 ** -4 * np.abs(v), 2.0 ** -10 * sv[None, :]) * (1 + 1e-6) + 1e-300
+    assert np.all(np.abs(deq - v) <= bound)
+    assert sv[3] == 0 and np.all(codes[:, 3] == 0)
+    col_max = np.argmax(np.abs(v), axis=0)
+    for c in range(24):
+        if c != 3:
+            assert abs(orc.e4m3_decode(codes[col_max[c], c])) == 448.0
+
+
+def test_integer_scores_brute_force():
+    rng = np.random.default_rng(5)
+    q8 = rng.integers(-127, 128, size=(7, 40)).astype(np.int8)
+    k8 = rng.integers(-127, 128, size=(9, 40)).astype(np.int8)
+    s = orc.integer_scores(q8, k8)
+    for i in range(7):
+        for j in range(9):
+            acc = 0
+            for c in range(40):
+                acc += int(q8[i, c]) * int(k8[j, c])
+            assert s[i, j] == acc
+
+
+def test_dequantized_scores_within_quantization_bound():
+    w = WORKLOADS["tiny"]
+    x = generate(w)
+    q, k = x["q"][0, 0], x["k"][0, 0]
+    r = orc.attention_head(q, k, x["v"][0, 0])
+    ks = orc.smooth_k(k, r["k_mean"]).astype(np.float64)
+    n = q.shape[0]
+    sq = r["q_scale"][np.arange(n) // orc.BLKQ].astype(np.float64)
+    sk = r["k_scale"][np.arange(n) // orc.BLKK].astype(np.float64)
+    deq = r["s_int"] * sq[:, None] * sk[None, :]
+    exact = q.astype(np.float64) @ ks.T
+    dq, dk = sq / 2, sk / 2
+    bound = (np.abs(q) @ np.ones(q.shape[1]))[:, None] * dk[None, :] \
+        + dq[:, None] * (np.abs(ks) @ np.ones(q.shape[1]))[None, :] \
+        + q.shape[1] * dq[:, None] * dk[None, :]
+    assert np.all(np.abs(deq - exact) <= bound * (1 + 1e-6))
+
+
+# ---------------------------------------------------------------- fp64 stages
+
+@pytest.mark.parametrize("n", [1, 5, 128, 200, 389])
+@pytest.mark.parametrize("causal", [False, True])
+def test_identity_quantizers_equal_textbook_attention(n, causal):
+    rng = np.random.default_rng(n)
+    q, k, v = (rng.standard_normal((n, 48)).astype(np.float32) for _ in range(3))
+    r = orc.attention_head(q, k, v, causal=causal, quantize=False)
+    ref = orc.reference_attention(q, k, v, causal=causal)
+    assert np.max(np.abs(r["out"] - ref)) <= 1e-12
+    # lse is that of the logits actually exponentiated; smoothing shifts it by
+    # q.mu/sqrt(d) per row, so compare it with smoothing switched off
+    r = orc.attention_head(q, k, v, causal=causal, quantize=False, smooth=False)
+    x = (q.astype(np.float64) @ k.astype(np.float64).T) / math.sqrt(48)
+    if causal:
+        x = np.where(np.arange(n)[None, :] > np.arange(n)[:, None], -np.inf, x)
+    lse = np.log(np.sum(np.exp(x), axis=1))
+    assert np.max(np.abs(r["lse"] - lse)) <= 1e-12
+
+
+def test_smoothing_invariance_in_exact_arithmetic():
+    rng = np.random.default_rng(7)
+    n, d = 300, 64
+    q, v = (rng.standard_normal((n, d)).astype(np.float32) for _ in range(2))
+    k = (rng.standard_normal((n, d)) + 5 * rng.standard_normal(d)[None, :]).astype(np.float32)
+    a = orc.attention_head(q, k, v, quantize=False, smooth=True)["out"]
+    b = orc.attention_head(q, k, v, quantize=False, smooth=False)["out"]
+    assert np.max(np.abs(a - b)) <= 1e-12
+    # a per-token shift of K is not a symmetry: the pin above is not vacuous
+    k2 = k + rng.standard_normal((n, 1)).astype(np.float32)
+    c = orc.attention_head(q, k2, v, quantize=False, smooth=True)["out"]
+    assert np.max(np.abs(c - a)) > 1e-3
+
+
+@pytest.mark.parametrize("quantize", [False, True])
+@pytest.mark.parametrize("causal", [False, True])
+def test_weights_rows_sum_to_one_and_causal_upper_triangle(quantize, causal):
+    rng = np.random.default_rng(8)
+    q, k = (rng.standard_normal((150, 32)).astype(np.float32) for _ in range(2))
+    p = orc.attention_weights(q, k, causal=causal, quantize=quantize)
+    assert np.max(np.abs(p.sum(axis=1) - 1)) <= 1e-12
+    if causal:
+        assert np.all(p[np.triu_indices(150, 1)] == 0)
+        assert p[0, 0] == 1.0
+
+
+def test_online_softmax_closed_form_across_tiles():
+    # logits that are exact multiples of ln 2 make every e4m3(448 * p) exact
+    n_kv, d = 200, 4
+    ln2 = math.log(2.0)
+    x = np.full((1, n_kv), -np.inf)
+    x[0, 0], x[0, 5], x[0, 70] = 0.0, -ln2, -3 * ln2           # tile 0, running max 0
+    x[0, 150], x[0, 199] = 2 * ln2, ln2                          # tile 1 raises the max
+    vals = np.array([1.0, -2.0, 0.5, 4.0])
+    vv = np.zeros((n_kv, d))
+    for j in (0, 5, 70, 150, 199):
+        vv[j] = vals * (1 + j % 3)
+    out, lse = orc.online_softmax_pv(x, vv, np.ones(d))
+    # tile 0: P8 = 448*[1, 1/2, 1/8]; tile 1 with m = 2 ln 2: 448*[1, 1/2]; tile 0 rescaled by 1/4
+    num = (448 * (vv[0] + vv[5] / 2 + vv[70] / 8)) / 4 + 448 * (vv[150] + vv[199] / 2)
+    l = (1 + 0.5 + 0.125) / 4 + 1.5
+    assert np.max(np.abs(out[0] - num / (448 * l))) <= 1e-12
+    assert abs(lse[0] - (2 * ln2 + math.log(l))) <= 1e-12
+
+
+def test_p_quantization_is_applied_per_block():
+    # exp(-0.1) * 448 = 405.36... rounds to 416 in e4m3; the unquantized sum keeps 0.9048
+    x = np.array([[0.0, -0.1]])
+    vv = np.array([[1.0], [3.0]])
+    out, _ = orc.online_softmax_pv(x, vv, np.ones(1))
+    p1 = math.exp(-0.1)
+    assert orc.e4m3_round(np.array([448 * p1]))[0] == 416.0
+    assert abs(out[0, 0] - (448 * 1 + 416 * 3) / (448 * (1 + p1))) <= 1e-12
+
+
+# ---------------------------------------------------------------- special cases
+
+def test_causal_first_row_and_single_token_return_dequantized_v():
+    w = WORKLOADS["tiny"]
+    x = generate(w)
+    q, k, v = x["q"][0, 1], x["k"][0, 1], x["v"][0, 1]
+    r = orc.attention_head(q, k, v, causal=True)
+    deq0 = orc.e4m3_decode(r["v8"][0]) * r["v_scale"].astype(np.float64)
+    assert np.array_equal(r["out"][0], deq0)
+    r1 = orc.attention_head(q[:1], k[:1], v[:1])
+    deq1 = orc.e4m3_decode(r1["v8"][0]) * r1["v_scale"].astype(np.float64)
+    assert np.array_equal(r1["out"][0], deq1)
+
+
+def test_identical_keys_give_mean_of_dequantized_v():
+    rng = np.random.default_rng(9)
+    n, d = 300, 64
+    q = rng.standard_normal((n, d)).astype(np.float32)
+    k = np.repeat(rng.standard_normal((1, d)).astype(np.float32), n, axis=0)
+    v = rng.standard_normal((n, d)).astype(np.float32)
+    r = orc.attention_head(q, k, v)
+    deq = orc.e4m3_decode(r["v8"]) * r["v_scale"].astype(np.float64)[None, :]
+    assert np.all(r["k8"] == 0)
+    assert np.max(np.abs(r["out"] - deq.mean(axis=0)[None, :])) <= 1e-12
+
+
+def test_gqa_equals_repeated_kv_heads():
+    rng = np.random.default_rng(10)
+    B, Hq, Hkv, N, d = 1, 4, 2, 130, 32
+    q = rng.standard_normal((B, Hq, N, d)).astype(np.float32)
+    k = rng.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    v = rng.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    a = orc.sage_attention(q, k, v, causal=True)
+    b = orc.sage_attention(q, np.repeat(k, 2, axis=1), np.repeat(v, 2, axis=1), causal=True)
+    assert np.array_equal(a, b)
+
+
+def test_varlen_equals_independent_sequences():
+    rng = np.random.default_rng(11)
+    lens = [70, 129, 1]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T, Hq, Hkv, d = cu[-1], 4, 2, 32
+    q = rng.standard_normal((T, Hq, d)).astype(np.float32)
+    k = rng.standard_normal((T, Hkv, d)).astype(np.float32)
+    v = rng.standard_normal((T, Hkv, d)).astype(np.float32)
+    out = orc.sage_attention(q, k, v, causal=True, cu_seqlens=cu)
+    for s0, s1 in zip(cu[:-1], cu[1:]):
+        one = orc.sage_attention(q[None, s0:s1].transpose(0, 2, 1, 3),
+                                 k[None, s0:s1].transpose(0, 2, 1, 3),
+                                 v[None, s0:s1].transpose(0, 2, 1, 3), causal=True)
+        assert np.array_equal(out[s0:s1], one[0].transpose(1, 0, 2))
+
+
+def test_row_subset_equals_full_rows():
+    w = WORKLOADS["tiny"]
+    x = generate(w)
+    q, k, v = x["q"][0, 0], x["k"][0, 0], x["v"][0, 0]
+    full = orc.attention_head(q, k, v, causal=True)
+    rows = np.array([0, 3, 127, 128, 255])
+    sub = orc.attention_head(q, k, v, causal=True, rows=rows)
+    assert np.array_equal(sub["out"], full["out"][rows])
+    assert np.array_equal(sub["lse"], full["lse"][rows])
+
+
+# ---------------------------------------------------------------- method accuracy
+
+def _metrics(o, ref):
+    o, ref = o.ravel(), ref.ravel()
+    cos = float(o @ ref / (np.linalg.norm(o) * np.linalg.norm(ref)))
+    rel_l1 = float(np.sum(np.abs(o - ref)) / np.sum(np.abs(ref)))
+    return cos, rel_l1
+
+
+def test_quantized_oracle_tracks_fp64_attention_on_tiny_workload():
+    w = WORKLOADS["tiny"]
+    x = generate(w)
+    out = orc.sage_attention(x["q"], x["k"], x["v"])
+    ref = np.stack([np.stack([orc.reference_attention(x["q"][0, h], x["k"][0, h], x["v"][0, h])
+                              for h in range(2)])])
+    cos, rel_l1 = _metrics(out, ref)
+    assert cos >= 0.999
+    assert rel_l1 <= 0.06
+
+
+def test_oracle_matches_its_committed_snapshot():
+    import json
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("make_golden", os.path.join(GOLDEN, "make_golden.py"))
+    mg = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mg)
+    with open(os.path.join(GOLDEN, "tiny_oracle_snapshot.json")) as f:
+        want = json.load(f)
+    got = mg.snapshot()
+    for hw, hg in zip(want["heads"], got["heads"]):
+        for key in ("q8_sha256", "k8_sha256", "v8_sha256", "s_int_sha256", "q_scale", "k_scale",
+                    "k_mean_first8"):
+            assert hw[key] == hg[key], key
+        assert np.max(np.abs(np.array(hw["out_rows"]) - np.array(hg["out_rows"]))) <= 1e-12
+        assert np.max(np.abs(np.array(hw["lse_rows"]) - np.array(hg["lse_rows"]))) <= 1e-12
