@@ -1,0 +1,174 @@
+/*
+ * sage.h - C ABI of the quantized attention forward for B200 (sm_100a).
+ *
+ * The method (SageAttention): K is smoothed by subtracting its per-channel mean,
+ * Q and K are quantized to INT8 per block, S = Q K^T runs on INT8 tensor cores
+ * with int32 accumulation, is dequantized, scaled and passed through an online
+ * softmax; P and V are quantized to FP8 e4m3 (V per channel) and P V is
+ * accumulated in two levels (per KV block, then into a running FP32 output).
+ * Sources: vibecrowd repo page "thu-ml--sageattention", How it works (INT8 QK^T,
+ * FP8 PV, two-level accumulation); glossary page "SageAttention(セージアテンション)",
+ * 概要 / 主な特徴・仕組み (K smoothing, INT8/FP8 per tensor); heatdrop review
+ * "2–5× attention speedups without the accuracy apology tour", Key highlights
+ * (GQA, variable sequence lengths); tutorial page "SageAttention终极指南",
+ * 基础使用示例 (sageattn(q, k, v, tensor_layout="HND", is_causal=False),
+ * shapes (batch, heads, seq_len, head_dim)).
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - Pointers are device memory owned by the caller unless marked "host".  The
+ *   library allocates no device memory and keeps no state between calls except
+ *   the device watchdog word read by sage_poll_device_status().
+ * - Work is enqueued on `stream` (a cudaStream_t); calls return once enqueued.
+ * - Errors: argument problems return SAGE_ERR_INVALID_ARGUMENT or
+ *   SAGE_ERR_UNSUPPORTED before anything is enqueued; a failed launch returns
+ *   SAGE_ERR_CUDA.  A kernel whose bounded wait runs out records
+ *   SAGE_ERR_DEVICE_TIMEOUT in the watchdog word and exits early (its outputs
+ *   are then undefined); the host reads that with sage_poll_device_status().
+ * - Input tensors q, k, v hold fp16 or bf16 values with a contiguous last
+ *   (head_dim) dimension.  Their other three dimensions are given as element
+ *   strides {stride_batch, stride_head, stride_token}: HND (B,H,N,d) and
+ *   NHD (B,N,H,d) are both expressed this way.  Varlen problems pack all
+ *   sequences along the token dimension (T_total, H, d); stride_batch is then
+ *   ignored and token t of sequence b is row cu_seqlens_host[b] + t.
+ * - Base pointers and the head/token strides must be 16-byte aligned in bytes.
+ *
+ * Quantized ("padded token space") buffers written by the quant entry points
+ * and read by sage_attn_fwd.  Let n_b be the length of sequence b,
+ * P_b = ceil(n_b / 128) * 128, off_b = sum_{b' < b} P_b' and T_pad = sum_b P_b
+ * (dense problems: n_b = seqlen for every b).  Padding entries are written as 0.
+ *   q8      int8  [Hq ][T_pad][d]       token t of seq b, head h at (h*T_pad + off_b + t)*d
+ *   q_scale float [Hq ][T_pad/128]      one scale per 128-token block of a sequence
+ *   k8      int8  [Hkv][T_pad][d]       smoothed K codes
+ *   k_scale float [Hkv][T_pad/64]       one scale per 64-token block of a sequence
+ *   k_mean  float [B  ][Hkv][d]         per-channel mean of K over the sequence
+ *   v8      uint8 [Hkv][d][T_pad]       e4m3 codes, transposed (token-contiguous)
+ *   v_scale float [B  ][Hkv][d]         per-channel V scale
+ * Dequantized values: q = q8 * q_scale, k - k_mean = k8 * k_scale,
+ * v = e4m3(v8) * v_scale.
+ */
+#ifndef SAGE_B200_H
+#define SAGE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sage_stream_t; /* the same handle as cudaStream_t */
+
+typedef enum {
+  SAGE_OK = 0,
+  SAGE_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size, misaligned, too small workspace */
+  SAGE_ERR_UNSUPPORTED = 2,      /* head_dim not 64/128, unknown dtype, device not sm_100 */
+  SAGE_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed */
+  SAGE_ERR_DEVICE_TIMEOUT = 4    /* a kernel's bounded wait ran out (see sage_poll_device_status) */
+} sage_status_t;
+
+typedef enum { SAGE_FP16 = 0, SAGE_BF16 = 1, SAGE_FP32 = 2 } sage_dtype_t;
+
+/* Problem description shared by all entry points. */
+typedef struct {
+  int batch;              /* B: dense batch size, or number of packed sequences (<= 1024) */
+  int heads_q;            /* Hq */
+  int heads_kv;           /* Hkv; Hq % Hkv == 0, query head h reads KV head h / (Hq/Hkv) */
+  int seqlen;             /* dense: tokens per sequence (>= 1); varlen: ignored */
+  int head_dim;           /* d: 64 or 128 */
+  sage_dtype_t dtype;     /* dtype of q, k, v: SAGE_FP16 or SAGE_BF16 */
+  const int32_t* cu_seqlens_host; /* host, NULL for dense; else [batch+1] prefix sums of the
+                                     packed sequence lengths, cu[0] = 0, non-decreasing */
+} sage_problem_t;
+
+/* Byte sizes of the quantized buffers and of the quantization workspaces. */
+typedef struct {
+  size_t q8, q_scale, k8, k_scale, k_mean, v8, v_scale;
+  size_t workspace_qk;    /* scratch needed by sage_quant_qk */
+  size_t workspace_v;     /* scratch needed by sage_quant_v */
+  size_t t_pad;           /* T_pad, the padded token count */
+} sage_sizes_t;
+
+/* Fill *sizes (host) for problem *p (host).  Pure host computation. */
+sage_status_t sage_buffer_sizes(const sage_problem_t* p, sage_sizes_t* sizes);
+
+/*
+ * sage_quant_qk - K smoothing and per-block INT8 quantization of Q and K.
+ * (glossary page "SageAttention(セージアテンション)", 主な特徴・仕組み: K smoothing;
+ *  vibecrowd page, How it works: INT8 quantization for QK^T.)
+ *   mu[c]  = fp32(sum_t k[t,c] in fp64 / n_b)              per (sequence, kv head)
+ *   k_s    = fp32(k - mu)
+ *   per block (Q: 128 tokens x d, K: 64 tokens x d of k_s):
+ *     a = max|x|;  s = fp32(a/127);  x8 = clamp(rint_even(fp32(x * fp32(127/a))), -127, 127)
+ *     (a == 0: s = 0, codes 0)
+ * Writes q8, q_scale, k8, k_scale, k_mean (layouts above).  `workspace` must
+ * hold sizes.workspace_qk bytes (fp64 per-block channel sums); its contents on
+ * entry do not matter.  Launches three kernels on `stream`.
+ */
+sage_status_t sage_quant_qk(const sage_problem_t* p,
+                            const void* q, const int64_t q_strides[3],
+                            const void* k, const int64_t k_strides[3],
+                            int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
+                            float* k_mean, void* workspace, size_t workspace_bytes,
+                            sage_stream_t stream);
+
+/*
+ * sage_quant_v - per-channel FP8 e4m3 quantization of V, written transposed.
+ * (vibecrowd page, How it works: FP8 for PV; glossary page, 概要: P and V in FP8.)
+ *   vmax[c] = max_t |v[t,c]| per (sequence, kv head);  sv = fp32(vmax/448)
+ *   v8 = e4m3_rne_satfinite(fp32(v * fp32(448/vmax)))   (vmax == 0: sv = 0, codes 0)
+ * Writes v8 and v_scale.  `workspace` must hold sizes.workspace_v bytes.
+ * Launches three kernels on `stream`.
+ */
+sage_status_t sage_quant_v(const sage_problem_t* p, const void* v, const int64_t v_strides[3],
+                           uint8_t* v8, float* v_scale, void* workspace, size_t workspace_bytes,
+                           sage_stream_t stream);
+
+/*
+ * sage_attn_fwd - the attention kernel (tcgen05 INT8 QK^T and FP8 PV, TMEM accumulators).
+ * (vibecrowd page, How it works; heatdrop review, The interesting bit and Key highlights.)
+ * For each query row i of sequence b, head h (KV head h/(Hq/Hkv)), over KV blocks of
+ * 128 keys in order:
+ *   x_j  = S_ij * q_scale * k_scale_j * sm_scale   (S_ij exact int32 from INT8 MMAs)
+ *   causal: x_j = -inf for j > i
+ *   m'   = max(m, max_j x_j);   P~_j = exp(x_j - m');   l = l e^{m-m'} + sum_j P~_j
+ *   P8   = e4m3(448 P~);  PV_blk = P8 V8 (FP32, fresh per block);  O = O e^{m-m'} + PV_blk
+ *   out  = O * v_scale / (448 l)           lse = m + ln(l)   (natural log)
+ * sm_scale <= 0 selects 1/sqrt(head_dim).  is_causal != 0 applies the mask above.
+ * out: written in out_dtype (SAGE_FP16, SAGE_BF16 or SAGE_FP32) with element
+ * strides out_strides {batch, head, token}, last dimension contiguous, the
+ * same packing rules as the inputs.  lse: NULL or float [Hq][T_pad], natural-log
+ * sum of exponentials of the smoothed, dequantized logits (padding rows unwritten).
+ * One kernel launch on `stream`.
+ */
+sage_status_t sage_attn_fwd(const sage_problem_t* p,
+                            const int8_t* q8, const float* q_scale,
+                            const int8_t* k8, const float* k_scale,
+                            const uint8_t* v8, const float* v_scale,
+                            float sm_scale, int is_causal,
+                            void* out, sage_dtype_t out_dtype, const int64_t out_strides[3],
+                            float* lse, sage_stream_t stream);
+
+/*
+ * sage_debug_qk_int32 - test hook: the exact int32 scores of one (sequence, query head).
+ * s_out: int32 [P_b][P_b] row-major, S[i][j] = sum_c q8[i][c] k8[j][c] over the padded
+ * rows of sequence `seq`, query head `head_q` and its KV head.  Uses the same
+ * TMA + tcgen05.mma kind::i8 + TMEM path as sage_attn_fwd.
+ */
+sage_status_t sage_debug_qk_int32(const sage_problem_t* p, const int8_t* q8, const int8_t* k8,
+                                  int seq, int head_q, int32_t* s_out, sage_stream_t stream);
+
+/*
+ * Synchronize `stream`, then read and clear the device watchdog word of the
+ * current device.  Returns SAGE_OK, SAGE_ERR_DEVICE_TIMEOUT or SAGE_ERR_CUDA.
+ */
+sage_status_t sage_poll_device_status(sage_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* sage_status_string(sage_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_B200_H */

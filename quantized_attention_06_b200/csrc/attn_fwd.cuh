@@ -1,0 +1,447 @@
+// attn_fwd.cuh - quantized attention forward on sm_100a tensor cores.
+//
+// Method (SageAttention): vibecrowd repo page "thu-ml--sageattention", How it
+// works (INT8 QK^T, FP8 PV, two-level accumulation for PV); heatdrop review
+// "2–5× attention speedups without the accuracy apology tour", The interesting
+// bit (two-level accumulation inside FP8 tensor cores) and Key highlights (GQA,
+// variable lengths); glossary page "SageAttention(セージアテンション)" (FlashAttention-
+// compatible online softmax).
+//
+// CTA = one (sequence, query head, pair of 128-row Q tiles).  12 warps in three
+// warpgroups; the producer warpgroup gives registers to the softmax warpgroups
+// (setmaxnreg: 128 x 40 + 256 x 232 = 384 x 168, the launch allocation):
+//   warp 0      TMA producer: both Q tiles once, then K / V tiles into 3-stage rings
+//   warp 1      TMEM owner and MMA issuer (one thread):
+//                 S_t  = Q8_t K8^T      tcgen05.mma kind::i8     -> TMEM s32 [128 x 128]
+//                 PV_t = P8_t V8       tcgen05.mma kind::f8f6f4 (A = P8 in TMEM) -> TMEM f32 [128 x d]
+//   warps 2-3   idle
+//   warps 4-7   softmax + correction for Q tile 0 (one thread per query row)
+//   warps 8-11  softmax + correction for Q tile 1
+// TMEM columns: [0,128) S/P of tile 0, [128,256) S/P of tile 1,
+//               [256,256+d) PV of tile 0, [384,384+d) PV of tile 1.
+// P8 of tile t is written over the first 32 columns of its S region (4 e4m3 per
+// column); the MMA that overwrites them with the next S is issued after the PV
+// MMA that reads them, and tcgen05.mma ops of one thread execute in issue order.
+//
+// Per KV tile j the softmax thread of query row i (log2 domain, u = x * log2 e):
+//   u_j   = S_ij * (q_scale * k_scale_j * sm_scale * log2 e)
+//   m'    = max(m, max_j u_j);  alpha = 2^(m - m')
+//   p_j   = 2^(u_j - m' + log2 448)   (= 448 * exp(x_j - x_max'))
+//   l     = l * alpha + sum_j p_j     (unquantized), P8_j = e4m3(p_j) -> TMEM
+//   O     = O * alpha + PV_blk        (PV_blk = P8 V8 in FP32, fresh each tile)
+//   out   = O * v_scale / l ;  lse = m' ln 2 + ln(l / 448)
+#pragma once
+
+#include <type_traits>
+
+#include "sage_device.cuh"
+#include "seq_table.cuh"
+
+namespace sage {
+
+constexpr int kAttnThreads = 384;
+constexpr int kAttnLaunchRegs = 168;  // 65536 / 384 rounded down to a multiple of 8
+constexpr int kProducerRegs = 40;
+constexpr int kSoftmaxRegs = 232;
+static_assert(128 * kProducerRegs + 256 * kSoftmaxRegs <= kAttnThreads * kAttnLaunchRegs,
+              "register split exceeds the launch allocation");
+constexpr int kKStages = 3;
+constexpr int kVStages = 3;
+constexpr float kLog2E = 1.4426950408889634f;
+constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
+constexpr float kLn448 = 6.104793232414985f;     // ln(448)
+
+struct AttnArgs {
+  const float* q_scale;  // [Hq][T_pad/128]
+  const float* k_scale;  // [Hkv][T_pad/64]
+  const float* v_scale;  // [B][Hkv][D]
+  void* out;
+  int out_dtype;  // 0 fp16, 1 bf16, 2 fp32
+  int64_t osb, osh, ost;
+  float* lse;  // [Hq][T_pad] or null
+  int hq, hkv, group;
+  float scale_log2;  // sm_scale * log2(e)
+  int causal;
+};
+
+template <int D>
+struct AttnSmem {
+  static constexpr int kTileQ = kBlkQ * D;      // bytes of one Q (or K) tile
+  static constexpr int kTileV = D * kKvTile;    // bytes of one V^T tile
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + 2 * kTileQ;
+  static constexpr int kVOff = kKOff + kKStages * kTileQ;
+  static constexpr int kBarOff = kVOff + kVStages * kTileV;
+  // barriers: q_full, k_full[3], k_empty[3], v_full[3], v_empty[3], s_full[2], p_full[2],
+  // pv_full[2], mma_done  -> 20 x 8 bytes, then the TMEM address slot
+  static constexpr int kNumBars = 20;
+  static constexpr int kSlotOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kSlotOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
+};
+
+__device__ __forceinline__ float i2f_exact(uint32_t s) {
+  // exact int32 -> fp32 for |s| < 2^22: place s in the mantissa of 1.5 * 2^23
+  return __int_as_float(static_cast<int>(s) + 0x4B400000) - 12582912.0f;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int D, class Seq>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                     const __grid_constant__ CUtensorMap tmap_k,
+                     const __grid_constant__ CUtensorMap tmap_v,
+                     const __grid_constant__ Seq seq, const __grid_constant__ AttnArgs a) {
+  using L = AttnSmem<D>;
+  constexpr uint32_t kSwizzle = (D == 128) ? 2u : 4u;  // UMMA layout type: 128B / 64B swizzle
+  constexpr uint32_t kSboQK = 8u * D;                  // 8 rows of D bytes
+  constexpr uint32_t kIdescS = idesc_i8(128, kKvTile);
+  constexpr uint32_t kIdescPV = idesc_e4m3_f32(128, D);
+  constexpr uint32_t kColS0 = 0, kColPV0 = 256;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::kBarOff;
+  auto bar_q = [&]() { return bar0; };
+  auto bar_kf = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto bar_ke = [&](int s) { return bar0 + 8u * (4 + s); };
+  auto bar_vf = [&](int s) { return bar0 + 8u * (7 + s); };
+  auto bar_ve = [&](int s) { return bar0 + 8u * (10 + s); };
+  auto bar_s = [&](int t) { return bar0 + 8u * (13 + t); };
+  auto bar_p = [&](int t) { return bar0 + 8u * (15 + t); };
+  auto bar_pv = [&](int t) { return bar0 + 8u * (17 + t); };
+  const uint32_t bar_done = bar0 + 8u * 19;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---------------------------------------------------------------- work item
+  int b, hq, pair;
+  {
+    int idx = blockIdx.x;
+    if constexpr (std::is_same<Seq, SeqDense>::value) {
+      const int nq = (seq_len(seq, 0) + kBlkQ - 1) / kBlkQ;
+      const int pairs = (nq + 1) / 2;
+      const int g = idx % a.group; idx /= a.group;
+      pair = idx % pairs; idx /= pairs;
+      const int hk = idx % a.hkv;
+      b = idx / a.hkv;
+      hq = hk * a.group + g;
+      if (a.causal) pair = pairs - 1 - pair;  // heaviest pairs first
+    } else {
+      int lo = 0, hi = seq.nseq - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (seq.cta[mid] <= idx) lo = mid; else hi = mid - 1;
+      }
+      while (lo + 1 < seq.nseq && seq.cta[lo + 1] <= idx) ++lo;
+      b = lo;
+      idx -= seq.cta[b];
+      const int nq = (seq_len(seq, b) + kBlkQ - 1) / kBlkQ;
+      const int pairs = (nq + 1) / 2;
+      const int g = idx % a.group; idx /= a.group;
+      pair = idx % pairs; idx /= pairs;
+      hq = idx * a.group + g;
+      if (a.causal) pair = pairs - 1 - pair;
+    }
+  }
+  const int hk = hq / a.group;
+  const int n = seq_len(seq, b);
+  const int off = seq_off(seq, b);
+  const int nq_tiles = (n + kBlkQ - 1) / kBlkQ;
+  const int nkv_all = (n + kKvTile - 1) / kKvTile;
+  int qt[2], nkv[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    qt[t] = 2 * pair + t;
+    nkv[t] = (qt[t] < nq_tiles) ? (a.causal ? qt[t] + 1 : nkv_all) : 0;
+  }
+  const int n_iter = max(nkv[0], nkv[1]);
+
+  // ---------------------------------------------------------------- set-up
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q(), 1);
+    for (int s = 0; s < kKStages; ++s) { mbar_init(bar_kf(s), 1); mbar_init(bar_ke(s), 1); }
+    for (int s = 0; s < kVStages; ++s) { mbar_init(bar_vf(s), 1); mbar_init(bar_ve(s), 1); }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_s(t), 1);
+      mbar_init(bar_p(t), 4);  // one arrival per softmax warp
+      mbar_init(bar_pv(t), 1);
+    }
+    mbar_init(bar_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool dead = watchdog_tripped();
+
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+   if (warp == 0) {
+    // ============================================================ TMA producer
+    if (lane == 0 && !dead) {
+      bool ok = true;
+      const int qbytes = (nkv[1] > 0 ? 2 : 1) * L::kTileQ;
+      mbar_arrive_expect_tx(bar_q(), qbytes);
+      for (int t = 0; t < 2; ++t)
+        if (nkv[t] > 0)
+          tma_load_2d(sbase + L::kQOff + t * L::kTileQ, &tmap_q, 0,
+                      hq * seq.t_pad + off + qt[t] * kBlkQ, bar_q());
+      int nk = 0, nv = 0;  // loads issued
+      for (int j = 0; j < n_iter && ok; ++j) {
+        const int ks = j % kKStages, vs = j % kVStages;
+        if (j >= kKStages) ok = mbar_wait(bar_ke(ks), ((j / kKStages) - 1) & 1, 0x101);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar_kf(ks), L::kTileQ);
+        tma_load_2d(sbase + L::kKOff + ks * L::kTileQ, &tmap_k, 0,
+                    hk * seq.t_pad + off + j * kKvTile, bar_kf(ks));
+        ++nk;
+        if (j >= kVStages) ok = mbar_wait(bar_ve(vs), ((j / kVStages) - 1) & 1, 0x102);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar_vf(vs), L::kTileV);
+        tma_load_2d(sbase + L::kVOff + vs * L::kTileV, &tmap_v, off + j * kKvTile, hk * D,
+                    bar_vf(vs));
+        ++nv;
+      }
+      // drain: the most recent load of every stage has landed before the CTA can exit
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bar_q(), 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
+      for (int jj = max(0, nk - kKStages); jj < nk; ++jj)
+        while (!mbar_try_wait(bar_kf(jj % kKStages), (jj / kKStages) & 1) &&
+               global_timer_ns() - t0 < kWaitLimitNs) {}
+      for (int jj = max(0, nv - kVStages); jj < nv; ++jj)
+        while (!mbar_try_wait(bar_vf(jj % kVStages), (jj / kVStages) & 1) &&
+               global_timer_ns() - t0 < kWaitLimitNs) {}
+    }
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (lane == 0 && !dead) {
+      // descriptors differ only in their start-address field (bits 0-13, address >> 4):
+      // keep one base per operand and add offsets at issue time
+      const uint64_t dq = sdesc_kmajor(sbase + L::kQOff, kSboQK, kSwizzle);
+      const uint64_t dk = sdesc_kmajor(sbase + L::kKOff, kSboQK, kSwizzle);
+      const uint64_t dv = sdesc_kmajor(sbase + L::kVOff, 1024u, 2u);
+      auto issue_s = [&](int t, int ks) {
+        const uint64_t aq = dq + static_cast<uint64_t>((t * L::kTileQ) >> 4);
+        const uint64_t bk = dk + static_cast<uint64_t>((ks * L::kTileQ) >> 4);
+        const uint32_t d_tmem = tmem + kColS0 + 128u * t;
+#pragma unroll
+        for (int s = 0; s < D / 32; ++s)
+          mma_i8_ss(d_tmem, aq + 2u * s, bk + 2u * s, kIdescS, s > 0 ? 1u : 0u);
+        tc_commit(bar_s(t));
+      };
+      auto issue_pv = [&](int t, int vs) {
+        const uint64_t bv = dv + static_cast<uint64_t>((vs * L::kTileV) >> 4);
+        const uint32_t d_tmem = tmem + kColPV0 + 128u * t;
+        const uint32_t a_tmem = tmem + kColS0 + 128u * t;
+#pragma unroll
+        for (int s = 0; s < kKvTile / 32; ++s)
+          mma_f8_ts(d_tmem, a_tmem + 8u * s, bv + 2u * s, kIdescPV, s > 0 ? 1u : 0u);
+        tc_commit(bar_pv(t));
+      };
+      bool ok = mbar_wait(bar_q(), 0, 0x201) && mbar_wait(bar_kf(0), 0, 0x202);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (nkv[t] > 0) issue_s(t, 0);
+        tc_commit(bar_ke(0));
+      }
+      for (int j = 0; j < n_iter && ok; ++j) {
+        const int vs = j % kVStages;
+        bool v_ready = false, k_ready = false;
+        const int jn = j + 1, ksn = jn % kKStages;
+        bool issued_next = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= nkv[t]) continue;
+          ok = mbar_wait(bar_p(t), j & 1, 0x203 + t);
+          if (ok && !v_ready) { ok = mbar_wait(bar_vf(vs), (j / kVStages) & 1, 0x205); v_ready = true; }
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(t, vs);
+          if (jn < nkv[t]) {
+            if (!k_ready) { ok = mbar_wait(bar_kf(ksn), (jn / kKStages) & 1, 0x206); k_ready = true; }
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(t, ksn);
+            issued_next = true;
+          }
+        }
+        if (!ok) break;
+        if (issued_next) tc_commit(bar_ke(ksn));
+        tc_commit(bar_ve(vs));
+      }
+      // every MMA issued by this thread has completed before TMEM is released
+      tc_commit(bar_done);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bar_done, 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
+    }
+   }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    // ============================================================ softmax + correction
+    const int t = (warp - 4) >> 2;  // Q tile of this warpgroup
+    const int quarter = warp & 3;   // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;
+    const int grow = qt[t] * kBlkQ + row;  // query index within the sequence
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + kColS0 + 128u * t;
+    const uint32_t tPV = tmem + lane_base + kColPV0 + 128u * t;
+
+    float o[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) o[c] = 0.0f;
+    float m = -INFINITY, l = 0.0f;
+    bool ok = !dead;
+    const float sq = (nkv[t] > 0) ? a.q_scale[static_cast<int64_t>(hq) * (seq.t_pad / kBlkQ) +
+                                              off / kBlkQ + qt[t]]
+                                  : 0.0f;
+    const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kBlkK) + off / kBlkK;
+
+    for (int j = 0; j < nkv[t] && ok; ++j) {
+      const float ck0 = sq * ksc[2 * j] * a.scale_log2;
+      const float ck1 = sq * ksc[2 * j + 1] * a.scale_log2;
+      const bool masked = (a.causal && j == qt[t]) || (j + 1) * kKvTile > n;
+      const int kv0 = j * kKvTile;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_s(t), j & 1, 0x301 + t));
+      if (!ok) break;
+      tc_fence_after();
+
+      // pass 1: row maximum of the integer scores in each 64-key half
+      int imax0 = INT_MIN, imax1 = INT_MIN;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tS + 32u * c, r);
+        tmem_wait_ld();
+        int mx = INT_MIN;
+        if (masked) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int key = kv0 + 32 * c + i;
+            const bool drop = key >= n || (a.causal && key > grow);
+            mx = max(mx, drop ? INT_MIN : static_cast<int>(r[i]));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx = max(mx, static_cast<int>(r[i]));
+        }
+        if (c < 2) imax0 = max(imax0, mx); else imax1 = max(imax1, mx);
+      }
+      const float mt = fmaxf(imax0 == INT_MIN ? -INFINITY : static_cast<float>(imax0) * ck0,
+                             imax1 == INT_MIN ? -INFINITY : static_cast<float>(imax1) * ck1);
+      const float m_new = fmaxf(m, mt);
+      const float alpha = ex2(m - m_new);
+      const float nbias = kLog2_448 - m_new;
+
+      // pass 2: p = 448 * 2^(u - m'), running sum, e4m3 P8 into TMEM over the S columns
+      float lt = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tS + 32u * c, r);
+        tmem_wait_ld();
+        const float ck = (c < 2) ? ck0 : ck1;
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float p[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            p[e] = ex2(fmaf(i2f_exact(r[4 * i + e]), ck, nbias));
+            if (masked) {
+              const int key = kv0 + 32 * c + 4 * i + e;
+              if (key >= n || (a.causal && key > grow)) p[e] = 0.0f;
+            }
+          }
+          lt += (p[0] + p[1]) + (p[2] + p[3]);
+          w[i] = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
+        }
+        tmem_st8(tS + 8u * c, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p(t));
+      l = l * alpha + lt;
+      m = m_new;
+
+      // two-level accumulation: O = alpha * O + PV_blk (PV_blk fresh in TMEM for this tile)
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_pv(t), j & 1, 0x303 + t));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tPV + 32u * c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[32 * c + i] = fmaf(o[32 * c + i], alpha, __uint_as_float(r[i]));
+      }
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    if (ok && nkv[t] > 0 && grow < n) {
+      const float inv_l = 1.0f / l;
+      const float* vs = a.v_scale + (static_cast<int64_t>(b) * a.hkv + hk) * D;
+      const int64_t orow = seq_base(seq, b, a.osb, a.ost) + hq * a.osh + static_cast<int64_t>(grow) * a.ost;
+      if (a.out_dtype == 2) {
+        float* dst = reinterpret_cast<float*>(a.out) + orow;
+#pragma unroll
+        for (int c = 0; c < D; c += 4) {
+          float4 v = make_float4(o[c] * vs[c] * inv_l, o[c + 1] * vs[c + 1] * inv_l,
+                                 o[c + 2] * vs[c + 2] * inv_l, o[c + 3] * vs[c + 3] * inv_l);
+          *reinterpret_cast<float4*>(dst + c) = v;
+        }
+      } else if (a.out_dtype == 1) {
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.out) + orow;
+#pragma unroll
+        for (int c = 0; c < D; c += 8) {
+          __align__(16) __nv_bfloat16 h8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) h8[i] = __float2bfloat16_rn(o[c + i] * vs[c + i] * inv_l);
+          *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<const uint4*>(h8);
+        }
+      } else {
+        __half* dst = reinterpret_cast<__half*>(a.out) + orow;
+#pragma unroll
+        for (int c = 0; c < D; c += 8) {
+          __align__(16) __half h8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) h8[i] = __float2half_rn(o[c + i] * vs[c + i] * inv_l);
+          *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<const uint4*>(h8);
+        }
+      }
+      if (a.lse != nullptr)
+        a.lse[static_cast<int64_t>(hq) * seq.t_pad + off + grow] =
+            m * 0.6931471805599453f + (logf(l) - kLn448);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace sage

@@ -1,0 +1,298 @@
+// quant.cuh - smoothing and quantization kernels (HBM-streaming, 16-byte vector loads).
+//
+// K smoothing and per-block INT8 quantization of Q and K follow the glossary
+// page "SageAttention(セージアテンション)" (概要, 主な特徴・仕組み) and the vibecrowd
+// repo page "thu-ml--sageattention" (How it works: INT8 QK^T, FP8 PV).
+//
+// Arithmetic is written with explicit IEEE round-to-nearest intrinsics
+// (__fsub_rn, __fmul_rn, __fdiv_rn, __float2int_rn, __ddiv_rn) so that no
+// contraction or approximate division can change a code.
+//
+// Kernels (one 256-thread CTA per block of tokens of one head):
+//   k_colsum   fp64 per-channel sums of K over each 128-token padded block
+//   k_mean     per (sequence, kv head): mu = fp32(sum / n)
+//   v_colmax   per-channel max |V| over each 128-token padded block
+//   v_finalize per (sequence, kv head): vmax, v_scale = vmax / 448
+//   quant_qk   Q blocks of 128 tokens and smoothed K blocks of 64 tokens -> int8 + scale
+//   quant_v    V -> e4m3 with per-channel scale, written token-contiguous (transposed)
+#pragma once
+
+#include "sage_device.cuh"
+#include "seq_table.cuh"
+
+namespace sage {
+
+constexpr int kQuantThreads = 256;
+
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// ------------------------------------------------------------------------- K stats
+template <typename T, int D, class Seq>
+__global__ void __launch_bounds__(kQuantThreads)
+k_colsum_kernel(const __grid_constant__ Seq seq, const T* __restrict__ k, int64_t sb, int64_t sh,
+                int64_t st, double* __restrict__ partial) {
+  constexpr int VPR = D / 8;               // 16-byte vectors per token row
+  constexpr int RG = kQuantThreads / VPR;  // rows handled in parallel
+  constexpr int IT = kPad / RG;
+  __shared__ double red[RG][D];
+  const int pb = blockIdx.x, h = blockIdx.y;
+  const SeqPos sp = locate(seq, pb * kPad, sb, st);
+  const int t0 = pb * kPad - sp.off;
+  const int vc = threadIdx.x % VPR, rg = threadIdx.x / VPR;
+  const T* src = k + sp.base + h * sh + vc * 8;
+  uint4 v[IT];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int t = t0 + rg + it * RG;
+    v[it] = (t < sp.n) ? ld_stream16(src + t * st) : make_uint4(0, 0, 0, 0);
+  }
+  double acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    float f[8];
+    unpack8<T>(v[it], f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] += static_cast<double>(f[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) red[rg][vc * 8 + i] = acc[i];
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += kQuantThreads) {
+    double s = 0.0;
+#pragma unroll 4
+    for (int g = 0; g < RG; ++g) s += red[g][c];
+    partial[(static_cast<int64_t>(h) * (seq.t_pad / kPad) + pb) * D + c] = s;
+  }
+}
+
+template <int D, class Seq>
+__global__ void __launch_bounds__(D)
+k_mean_kernel(const __grid_constant__ Seq seq, const double* __restrict__ partial, int hkv,
+              float* __restrict__ k_mean) {
+  const int b = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
+  const int n = seq_len(seq, b);
+  const int blk0 = seq_off(seq, b) / kPad;
+  const int nblk = (n + kPad - 1) / kPad;
+  const double* p = partial + (static_cast<int64_t>(h) * (seq.t_pad / kPad) + blk0) * D + c;
+  double s = 0.0;
+  for (int i = 0; i < nblk; ++i) s += p[static_cast<int64_t>(i) * D];
+  const float mu = (n > 0) ? __double2float_rn(__ddiv_rn(s, static_cast<double>(n))) : 0.0f;
+  k_mean[(static_cast<int64_t>(b) * hkv + h) * D + c] = mu;
+}
+
+// ------------------------------------------------------------------------- V stats
+template <typename T, int D, class Seq>
+__global__ void __launch_bounds__(kQuantThreads)
+v_colmax_kernel(const __grid_constant__ Seq seq, const T* __restrict__ v, int64_t sb, int64_t sh,
+                int64_t st, float* __restrict__ partial) {
+  constexpr int VPR = D / 8;
+  constexpr int RG = kQuantThreads / VPR;
+  constexpr int IT = kPad / RG;
+  __shared__ float red[RG][D];
+  const int pb = blockIdx.x, h = blockIdx.y;
+  const SeqPos sp = locate(seq, pb * kPad, sb, st);
+  const int t0 = pb * kPad - sp.off;
+  const int vc = threadIdx.x % VPR, rg = threadIdx.x / VPR;
+  const T* src = v + sp.base + h * sh + vc * 8;
+  uint4 x[IT];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int t = t0 + rg + it * RG;
+    x[it] = (t < sp.n) ? ld_stream16(src + t * st) : make_uint4(0, 0, 0, 0);
+  }
+  float mx[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx[i] = 0.0f;
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    float f[8];
+    unpack8<T>(x[it], f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], fabsf(f[i]));
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) red[rg][vc * 8 + i] = mx[i];
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += kQuantThreads) {
+    float m = 0.0f;
+    for (int g = 0; g < RG; ++g) m = fmaxf(m, red[g][c]);
+    partial[(static_cast<int64_t>(h) * (seq.t_pad / kPad) + pb) * D + c] = m;
+  }
+}
+
+template <int D, class Seq>
+__global__ void __launch_bounds__(D)
+v_finalize_kernel(const __grid_constant__ Seq seq, const float* __restrict__ partial, int hkv,
+                  float* __restrict__ vmax_out, float* __restrict__ v_scale) {
+  const int b = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
+  const int n = seq_len(seq, b);
+  const int blk0 = seq_off(seq, b) / kPad;
+  const int nblk = (n + kPad - 1) / kPad;
+  const float* p = partial + (static_cast<int64_t>(h) * (seq.t_pad / kPad) + blk0) * D + c;
+  float m = 0.0f;
+  for (int i = 0; i < nblk; ++i) m = fmaxf(m, p[static_cast<int64_t>(i) * D]);
+  const int64_t o = (static_cast<int64_t>(b) * hkv + h) * D + c;
+  vmax_out[o] = m;
+  v_scale[o] = (m > 0.0f) ? __fdiv_rn(m, 448.0f) : 0.0f;
+}
+
+// ------------------------------------------------------------------------- Q/K INT8
+struct QKQuantArgs {
+  const void* q;
+  const void* k;
+  int64_t qsb, qsh, qst, ksb, ksh, kst;
+  int8_t* q8;
+  float* q_scale;
+  int8_t* k8;
+  float* k_scale;
+  const float* k_mean;
+  int hq, hkv;
+  int nq_blocks;  // hq * t_pad / 128 (the first CTAs); the rest are K blocks
+};
+
+__device__ __forceinline__ float block_max_256(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float m = red[0];
+#pragma unroll
+  for (int i = 1; i < kQuantThreads / 32; ++i) m = fmaxf(m, red[i]);
+  return m;
+}
+
+__device__ __forceinline__ uint32_t pack_i8x4(int a, int b, int c, int d) {
+  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
+         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
+}
+
+__device__ __forceinline__ int quant_i8(float x, float r) {
+  const int q = __float2int_rn(__fmul_rn(x, r));
+  return max(-127, min(127, q));
+}
+
+template <typename T, int D, class Seq>
+__global__ void __launch_bounds__(kQuantThreads)
+quant_qk_kernel(const __grid_constant__ Seq seq, const __grid_constant__ QKQuantArgs a) {
+  constexpr int VPR = D / 8;
+  constexpr int RG = kQuantThreads / VPR;
+  constexpr int ITQ = kBlkQ / RG;  // 8 (d=128) or 4 (d=64)
+  __shared__ float red[kQuantThreads / 32];
+  const bool isq = static_cast<int>(blockIdx.x) < a.nq_blocks;
+  const int rows = isq ? kBlkQ : kBlkK;
+  const int per_head = seq.t_pad / rows;
+  const int local = isq ? blockIdx.x : blockIdx.x - a.nq_blocks;
+  const int h = local / per_head, pb = local % per_head;
+  const int tp = pb * rows;
+  const int64_t sb = isq ? a.qsb : a.ksb, sh = isq ? a.qsh : a.ksh, st = isq ? a.qst : a.kst;
+  const SeqPos sp = locate(seq, tp, sb, st);
+  const int t0 = tp - sp.off;
+  const int vc = threadIdx.x % VPR, rg = threadIdx.x / VPR;
+  const T* src = reinterpret_cast<const T*>(isq ? a.q : a.k) + sp.base + h * sh + vc * 8;
+
+  float mu[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mu[i] = 0.0f;
+  if (!isq) {
+    const float* m = a.k_mean + (static_cast<int64_t>(sp.b) * a.hkv + h) * D + vc * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mu[i] = m[i];
+  }
+  const int iters = rows / RG;
+  float x[ITQ][8];
+  float amax = 0.0f;
+#pragma unroll
+  for (int it = 0; it < ITQ; ++it) {
+    const int t = t0 + rg + it * RG;
+    const bool valid = it < iters && t < sp.n;
+    uint4 v = valid ? ld_stream16(src + t * st) : make_uint4(0, 0, 0, 0);
+    float f[8];
+    unpack8<T>(v, f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      x[it][i] = valid ? (isq ? f[i] : __fsub_rn(f[i], mu[i])) : 0.0f;
+      amax = fmaxf(amax, fabsf(x[it][i]));
+    }
+  }
+  amax = block_max_256(amax, red);
+  const float s = (amax > 0.0f) ? __fdiv_rn(amax, 127.0f) : 0.0f;
+  const float r = (amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
+  int8_t* dst = (isq ? a.q8 : a.k8) + (static_cast<int64_t>(h) * seq.t_pad + tp) * D + vc * 8;
+#pragma unroll
+  for (int it = 0; it < ITQ; ++it) {
+    if (it < iters) {
+      const int rr = rg + it * RG;
+      uint2 o;
+      o.x = pack_i8x4(quant_i8(x[it][0], r), quant_i8(x[it][1], r), quant_i8(x[it][2], r),
+                      quant_i8(x[it][3], r));
+      o.y = pack_i8x4(quant_i8(x[it][4], r), quant_i8(x[it][5], r), quant_i8(x[it][6], r),
+                      quant_i8(x[it][7], r));
+      *reinterpret_cast<uint2*>(dst + static_cast<int64_t>(rr) * D) = o;
+    }
+  }
+  if (threadIdx.x == 0) (isq ? a.q_scale : a.k_scale)[static_cast<int64_t>(h) * per_head + pb] = s;
+}
+
+// ------------------------------------------------------------------------- V e4m3
+struct VQuantArgs {
+  const void* v;
+  int64_t sb, sh, st;
+  const float* vmax;  // [B][Hkv][D]
+  uint8_t* v8;        // [Hkv][D][T_pad]
+  int hkv;
+};
+
+template <typename T, int D, class Seq>
+__global__ void __launch_bounds__(kQuantThreads)
+quant_v_kernel(const __grid_constant__ Seq seq, const __grid_constant__ VQuantArgs a) {
+  constexpr int VPR = D / 8;
+  constexpr int RG = kQuantThreads / VPR;
+  constexpr int IT = kPad / RG;
+  constexpr int LD = kPad + 16;  // padded smem row (bytes) of the transposed tile
+  __shared__ __align__(16) uint8_t tile[D][LD];
+  const int pb = blockIdx.x, h = blockIdx.y;
+  const SeqPos sp = locate(seq, pb * kPad, a.sb, a.st);
+  const int t0 = pb * kPad - sp.off;
+  const int vc = threadIdx.x % VPR, rg = threadIdx.x / VPR;
+  const T* src = reinterpret_cast<const T*>(a.v) + sp.base + h * a.sh + vc * 8;
+  float r[8];
+  {
+    const float* vm = a.vmax + (static_cast<int64_t>(sp.b) * a.hkv + h) * D + vc * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] = (vm[i] > 0.0f) ? __fdiv_rn(448.0f, vm[i]) : 0.0f;
+  }
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int rr = rg + it * RG;
+    const int t = t0 + rr;
+    const bool valid = t < sp.n;
+    const uint4 v = valid ? ld_stream16(src + t * a.st) : make_uint4(0, 0, 0, 0);
+    float f[8];
+    unpack8<T>(v, f);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const uint32_t two = valid ? e4m3x2(__fmul_rn(f[i], r[i]), __fmul_rn(f[i + 1], r[i + 1])) : 0u;
+      tile[vc * 8 + i][rr] = static_cast<uint8_t>(two & 0xFFu);
+      tile[vc * 8 + i + 1][rr] = static_cast<uint8_t>(two >> 8);
+    }
+  }
+  __syncthreads();
+  // each channel row of the tile is 128 contiguous output bytes: 8 threads x 16 B
+  uint8_t* dst = a.v8 + static_cast<int64_t>(h) * D * seq.t_pad + pb * kPad;
+  for (int i = threadIdx.x; i < D * 8; i += kQuantThreads) {
+    const int c = i >> 3, j = i & 7;
+    const uint4 w = *reinterpret_cast<const uint4*>(&tile[c][j * 16]);
+    *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(c) * seq.t_pad + j * 16) = w;
+  }
+}
+
+}  // namespace sage

@@ -1,0 +1,183 @@
+"""GPU parity of sage_attn_fwd against the oracle.
+
+Bars (GPU vs oracle, both with the same quantization): max-abs error <= 2e-3 and
+cosine similarity >= 0.9999 on fp32 output; lse within 1e-3.  Small cases are
+compared element by element on every row; full-size workloads on sampled rows
+(first and last tiles included) of several (sequence, head) pairs.  fp16 / bf16
+outputs are compared against the oracle rounded to that dtype, with one extra
+unit in the last place of the output allowed."""
+
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from quantized_attention_06_b200 import api
+from quantized_attention_06_b200.inputs import WORKLOADS, Workload, generate, sweep_workload
+
+from _helpers import MAX_ABS, MIN_COS, from_device_out, metrics, padded_offsets, run_gpu, seq_views
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_rows(x, w, causal, pairs):
+    """{(b, h): (rows, out, lse)} for the requested (b, h, rows) triples."""
+    g = w.heads_q // w.heads_kv
+    views = {b: (qb, kb, vb) for b, qb, kb, vb, _ in seq_views(x, w.varlen)}
+    res = {}
+    for b, h, rows in pairs:
+        qb, kb, vb = views[b]
+        r = orc.attention_head(qb[h], kb[h // g], vb[h // g], causal=causal, rows=rows)
+        res[(b, h)] = (r["rows"], r["out"], r["lse"])
+    return res
+
+
+def _gpu_rows(out_np, lse_np, x, w, b, h, rows):
+    lens = [int(n) for n in x["seqlens"]] if w.varlen else [w.seqlen] * w.batch
+    offs, _ = padded_offsets(lens)
+    if w.varlen:
+        s0 = int(x["cu_seqlens"][b])
+        o = out_np[s0 + rows, h]
+    else:
+        o = out_np[b, h, rows]
+    return o, lse_np[h, offs[b] + rows]
+
+
+def _check(x, w, causal, pairs, out_dtype=torch.float32):
+    z, out, lse = run_gpu(x, w.dtype, w.layout, w.varlen, causal, out_dtype=out_dtype)
+    out_np = from_device_out(out, w.layout, w.varlen)
+    lse_np = lse.cpu().numpy()
+    ref = _oracle_rows(x, w, causal, pairs)
+    for (b, h), (rows, o_ref, lse_ref) in ref.items():
+        o_gpu, l_gpu = _gpu_rows(out_np, lse_np, x, w, b, h, rows)
+        if out_dtype == torch.float32:
+            mx, cos, _ = metrics(o_gpu, o_ref)
+            assert mx <= MAX_ABS, (b, h, mx)
+        else:
+            o_ref_r = torch.from_numpy(o_ref).to(out_dtype).double().numpy()
+            ulp = np.abs(o_ref_r) * (2.0 ** -8 if out_dtype == torch.bfloat16 else 2.0 ** -11)
+            assert np.all(np.abs(o_gpu - o_ref_r) <= MAX_ABS + ulp), (b, h)
+            _, cos, _ = metrics(o_gpu, o_ref)
+        assert cos >= MIN_COS, (b, h, cos)
+        assert np.max(np.abs(l_gpu - lse_ref)) <= 1e-3, (b, h)
+    return out_np
+
+
+def _all_pairs(x, w):
+    lens = [int(n) for n in x["seqlens"]] if w.varlen else [w.seqlen] * w.batch
+    return [(b, h, None) for b in range(len(lens)) if lens[b] > 0 for h in range(w.heads_q)]
+
+
+SMALL = [
+    WORKLOADS["tiny"],
+    Workload("r1", 1, 2, 1, 1, 64, "fp16", "HND", seed=6),
+    Workload("r63", 2, 4, 2, 63, 128, "bf16", "NHD", seed=5),
+    Workload("r129", 1, 2, 2, 129, 128, "fp16", "HND", seed=10),
+    Workload("r200", 1, 3, 3, 200, 64, "bf16", "HND", seed=7, tail_frac=0.02, tail_scale=20.0),
+    Workload("r383", 2, 2, 2, 383, 128, "fp16", "NHD", seed=8, k_offset_sigma=4.0),
+    Workload("r640", 1, 4, 1, 640, 128, "bf16", "HND", seed=11),
+    Workload("vl", 5, 4, 2, 700, 128, "bf16", "NHD", seed=9, varlen=True, varlen_range=(1, 700),
+             varlen_count=5),
+    Workload("vl64", 4, 6, 3, 600, 64, "fp16", "NHD", seed=12, varlen=True, varlen_range=(100, 600),
+             varlen_count=4),
+]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_attention_small_all_rows(w, causal):
+    x = generate(w)
+    pairs = [(b, h, np.arange(qb.shape[1])) for b, qb, _, _, _ in seq_views(x, w.varlen)
+             if qb.shape[1] > 0 for h in range(w.heads_q)]
+    _check(x, w, causal, pairs)
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float16, torch.bfloat16])
+def test_attention_half_outputs(out_dtype):
+    w = SMALL[5]
+    x = generate(w)
+    pairs = [(b, h, np.arange(w.seqlen)) for b in range(w.batch) for h in range(w.heads_q)]
+    _check(x, w, True, pairs, out_dtype=out_dtype)
+
+
+def test_attention_varlen_with_empty_sequence():
+    w = replace(WORKLOADS["gqa_varlen"], name="vl_empty")
+    x = generate(w, seqlens=[300, 0, 129, 1])
+    pairs = [(b, h, np.arange(n)) for b, n in enumerate([300, 0, 129, 1]) if n > 0
+             for h in (0, 7, 31)]
+    _check(x, w, True, pairs)
+
+
+def _sample_rows(n, k=1024):
+    head = np.arange(min(n, 256))
+    tail = np.arange(max(0, n - 256), n)
+    mid = np.linspace(0, n - 1, k).astype(np.int64)
+    return np.unique(np.concatenate([head, mid, tail]))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_prefill(causal):
+    w = WORKLOADS["prefill"]
+    x = generate(w)
+    pairs = [(b, h, np.arange(w.seqlen)) for b, h in ((0, 0), (1, 13), (2, 31), (3, 7))]
+    _check(x, w, causal, pairs)
+
+
+@pytest.mark.parametrize("n", [4096, 32768])
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_sweep_sampled(n, causal):
+    w = sweep_workload(n)
+    x = generate(w)
+    pairs = [(0, h, _sample_rows(n)) for h in (0, 9, 22, 31)]
+    _check(x, w, causal, pairs)
+
+
+def test_attention_dit_sampled():
+    w = WORKLOADS["dit"]
+    x = generate(w)
+    pairs = [(b, h, _sample_rows(w.seqlen)) for b, h in ((0, 0), (0, 47), (1, 20), (1, 33))]
+    _check(x, w, False, pairs)
+
+
+def test_attention_gqa_varlen_sampled():
+    w = WORKLOADS["gqa_varlen"]
+    x = generate(w)
+    lens = [int(n) for n in x["seqlens"]]
+    pairs = [(b, h, _sample_rows(lens[b], 512)) for b in (0, 3, 7) for h in (0, 5, 31)]
+    _check(x, w, True, pairs)
+
+
+def test_gqa_equals_repeated_kv_on_gpu():
+    w = Workload("gqa", 1, 8, 2, 300, 128, "bf16", "HND", seed=13)
+    x = generate(w)
+    _, out_a, _ = run_gpu(x, w.dtype, w.layout, False, True)
+    x2 = dict(x, k=np.repeat(x["k"], 4, axis=1), v=np.repeat(x["v"], 4, axis=1))
+    _, out_b, _ = run_gpu(x2, w.dtype, w.layout, False, True)
+    assert torch.equal(out_a, out_b)
+
+
+def test_layouts_agree_on_gpu():
+    w = Workload("lay", 2, 4, 4, 333, 64, "fp16", "HND", seed=14)
+    x = generate(w)
+    _, out_h, _ = run_gpu(x, w.dtype, "HND", False, False)
+    _, out_n, _ = run_gpu(x, w.dtype, "NHD", False, False)
+    assert torch.equal(out_h, out_n.permute(0, 2, 1, 3))
+
+
+@pytest.mark.parametrize("name", ["tiny", "prefill"])
+def test_accuracy_against_full_precision(name):
+    """The kernel adds no error beyond the method: its fp64-attention metrics match
+    the oracle's own (cos >= 0.999 holds for these N(0,1) workloads)."""
+    w = WORKLOADS[name]
+    x = generate(w)
+    _, out, _ = run_gpu(x, w.dtype, w.layout, False, False)
+    o = from_device_out(out, w.layout, False)
+    for b, h in ((0, 0), (0, w.heads_q - 1)):
+        ref = orc.reference_attention(x["q"][b, h], x["k"][b, h], x["v"][b, h])
+        orc_out = orc.attention_head(x["q"][b, h], x["k"][b, h], x["v"][b, h])["out"]
+        _, cos_g, rl_g = metrics(o[b, h], ref)
+        _, cos_o, rl_o = metrics(orc_out, ref)
+        assert cos_g >= 0.999
+        assert abs(rl_g - rl_o) <= 0.1 * rl_o
