@@ -1,0 +1,332 @@
+"""Benchmark: quantized attention forward (INT8 QK^T, FP8 PV) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--n N] [--causal]
+
+Workload (default): the kernel-sweep configuration at its longest length,
+B=1, H=32, N=32768, d=128, fp16, HND, non-causal, seeded synthetic inputs
+(Q, V ~ N(0,1); K ~ N(0,1) plus a per-channel offset ~ N(0, 3^2)).
+
+A step is one pass of the whole path on device-resident inputs: sage_quant_qk
+(K mean, Q/K INT8), sage_quant_v (V e4m3) and sage_attn_fwd.  TOPS =
+4*B*H*N^2*d / time (halved when causal).  Inputs (3 x 256 MiB) exceed the
+126 MB L2, so no flush is needed between steps.  Rank 0 prints one JSON line.
+
+Multi-GPU (torchrun): every rank runs its own copy of the workload (independent
+problems, no data-path collective; weak scaling); the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "attention TOPS at hd128, seq 1K–32K (1×B200); % of INT8/FP8 tensor peak"
+UNIT = "TOPS"
+NOMINAL_INT8_OVER_BF16 = 2.0  # 4.5 POPS dense INT8/FP8 vs 2.25 PFLOP/s dense bf16 (datasheet ratio)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="sage", choices=["sage", "reference"])
+    ap.add_argument("--n", type=int, default=32768)
+    ap.add_argument("--causal", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=1536)
+    return ap.parse_args()
+
+
+def workload(args):
+    from quantized_attention_06_b200.inputs import sweep_workload
+    return sweep_workload(args.n)
+
+
+def config(w, args, n_gpus):
+    return {"workload": f"sweep B={w.batch} H={w.heads_q} N={w.seqlen} d={w.head_dim} "
+                        f"{w.dtype} {w.layout} {'causal' if args.causal else 'non-causal'}",
+            "batch": w.batch, "heads": w.heads_q, "seq_len": w.seqlen, "head_dim": w.head_dim,
+            "causal": bool(args.causal), "layout": w.layout, "n_gpus": n_gpus,
+            "l2": "inputs (3 x 256 MiB) larger than the 126 MB L2; no flush",
+            "step": "sage_quant_qk + sage_quant_v + sage_attn_fwd"}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p["bf16_tflops"], p.get("bf16_tflops_sustained"), p.get("hbm_gbs"), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def cpu_sample(w, args, rows):
+    """Time the oracle on a bounded sample: one head's quantization plus `rows`
+    evenly spaced query rows against all keys.  Returns (TOPS, seconds, sample)."""
+    import oracle as orc
+    from quantized_attention_06_b200.inputs import generate
+    x = generate(w)
+    q, k, v = x["q"][0, 0], x["k"][0, 0], x["v"][0, 0]
+    sel = np.linspace(0, w.seqlen - 1, rows).astype(np.int64)
+    t0 = time.perf_counter()
+    orc.attention_head_kernel_precision(q, k, v, causal=args.causal, rows=sel)
+    dt = time.perf_counter() - t0
+    n_keys = (sel + 1).sum() if args.causal else rows * w.seqlen
+    ops = 4.0 * n_keys * w.head_dim
+    sample = (f"head 0 quantization (Q, K, V) plus {rows} evenly spaced query rows against "
+              f"{'their causal prefix' if args.causal else f'all {w.seqlen} keys'}")
+    return ops / dt / 1e12, dt, sample
+
+
+def threads_used():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] + [1])
+    except Exception:
+        return 1
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    w = workload(args)
+    times = []
+    for i in range(args.warmup + args.steps):
+        tops, dt, sample = cpu_sample(w, args, max(8, args.cpu_rows // 4))
+        if i >= args.warmup:
+            times.append(tops)
+    val = statistics.median(times)
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (P8 decision fp32)",
+            "data": "synthetic", "config": config(w, args, world),
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads_used(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+class Clocks:
+    """nvidia-smi sampler running while the timed region runs."""
+
+    def __init__(self, dev_index):
+        self.dev = dev_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            self.proc.wait()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                    power.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        load = [s for s in sm if mx and s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+def run_sage(args):
+    import torch
+    import torch.distributed as dist
+
+    from quantized_attention_06_b200 import api
+    from quantized_attention_06_b200.inputs import generate
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+
+    w = workload(args)
+    x = generate(w)
+    host = {n: torch.from_numpy(x[n]).to(torch.float16).pin_memory() for n in ("q", "k", "v")}
+    del x
+    q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
+    p = api.Problem.from_tensors(q, k, "HND")
+    z = api.Quantized(p, "HND")
+    ws_qk = torch.empty(max(1, p.sizes.workspace_qk // 8), dtype=torch.float64, device=dev)
+    ws_v = torch.empty(max(1, p.sizes.workspace_v // 4), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    launches_per_step = 7  # k_colsum, k_mean, quant_qk, v_colmax, v_finalize, quant_v, attn
+
+    def step(ev=None):
+        api.quant_qk(q, k, "HND", problem=p, out=z, workspace=ws_qk)
+        api.quant_v(v, z, workspace=ws_v)
+        if ev is not None:
+            ev[0].record(stream)
+        api.attn_fwd(z, is_causal=args.causal, out=out)
+        if ev is not None:
+            ev[1].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    assert api.poll_device_status() == 0
+
+    # ---- whole-step timing (device events, max over ranks)
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        barrier()
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(attn_ev[i])
+        t_end.record(stream)
+        barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
+    if world > 1:
+        tt = torch.tensor([total_ms, statistics.mean(attn_ms)], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms, attn_mean = tt.tolist()
+    else:
+        attn_mean = statistics.mean(attn_ms)
+    assert api.poll_device_status() == 0
+
+    ops = w.ops(args.causal)
+    ms_per_step = total_ms / args.steps
+    value = ops * world / (ms_per_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        e_steps = max(2, args.steps // 2)
+
+        def e2e_step():
+            qd, kd, vd = (host[n].to(dev, non_blocking=True) for n in ("q", "k", "v"))
+            o = api.sageattn(qd, kd, vd, tensor_layout="HND", is_causal=args.causal)
+            host_out.copy_(o, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        e_ms = e0.elapsed_time(e1) / e_steps
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = tt.item()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        e2e = {"value": ops * world / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out.numel() * out.element_size(),
+               "ms_per_step": e_ms}
+
+    bf16, bf16_sus, _, src = peaks()
+    peak = bf16 * NOMINAL_INT8_OVER_BF16
+    achieved = ops / (attn_mean * 1e-3) / 1e12
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            tr = json.load(f)
+        import hashlib
+        src_hash = hashlib.sha256(open(os.path.join(ROOT, "quantized_attention_06_b200", "csrc",
+                                                    "attn_fwd.cuh"), "rb").read()).hexdigest()[:16]
+        if tr.get("source_sha16") == src_hash and tr.get("workload_n") == w.seqlen:
+            traffic = tr.get("bytes_per_launch")
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8 QK / e4m3 PV (fp32 softmax)",
+            "data": "synthetic", "config": config(w, args, world),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "sage_attn_fwd_kernel", "ms_per_launch": attn_mean,
+                         "peak_source": f"{src} bf16 burst {bf16} x nominal INT8/FP8:bf16 ratio 2",
+                         "frac_of_sustained": (achieved / (bf16_sus * NOMINAL_INT8_OVER_BF16)
+                                               if bf16_sus else None),
+                         "frac_of_datasheet_4500": achieved / 4500.0},
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+        }
+        if world == 1:
+            tops, dt, sample = cpu_sample(w, args, args.cpu_rows)
+            line["cpu_baseline"] = {"value": tops, "unit": UNIT, "cores": threads_used(),
+                                    "kind": "oracle", "sample": sample, "seconds": dt}
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_sage(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -19,7 +19,12 @@ What it computes, stage by stage, for one (sequence, query head) with its KV hea
    block, then added into the running output: two-level accumulation
    (vibecrowd page, How it works; heatdrop review, Key highlights).
 
-Everything after the integer scores is done in float64.
+Everything after the integer scores is done in float64, with one exception
+kept apart in ``attention_head_kernel_precision``: P8 is an integer code decided
+by floating point, so for GPU parity that decision is taken with the kernel's
+own fp32 steps (fp32 logits and running max, t = fma(S, ck, log2 448 - m'),
+the documented fp32 exp2 algorithm, e4m3 rounding); l, the rescale factors, PV
+and the output stay fp64.  ``attention_head`` is the all-fp64 definition.
 
 Readings where the pages are silent (each is listed in the design doc):
 
@@ -53,6 +58,8 @@ __all__ = [
     "k_channel_mean", "smooth_k", "quantize_int8_blocks", "quantize_v_e4m3",
     "integer_scores", "online_softmax_pv", "attention_head", "sage_attention",
     "reference_attention", "attention_weights",
+    "LOG2E_F32", "LOG2_448_F32", "EXP2_COEF_F32", "fma_f32", "exp2_f32", "kernel_scale_log2",
+    "online_softmax_pv_fp32_decision", "attention_head_kernel_precision",
 ]
 
 BLKQ = 128        # tokens per Q quantization block
@@ -331,3 +338,151 @@ def reference_attention(q, k, v, *, causal=False, sm_scale=None) -> np.ndarray:
     x = x - np.max(x, axis=1, keepdims=True)
     p = np.exp(x)
     return (p @ v) / np.sum(p, axis=1, keepdims=True)
+
+
+# --------------------------------------------------------------------------
+# The P8 decision taken in the kernel's precision
+# --------------------------------------------------------------------------
+# P8 is an integer code decided by floating point, so for parity both sides take
+# that decision with the same fp32 arithmetic: logits u = S * ck in the log2
+# domain, the running max m' over 64-key halves, t = fma(S, ck, log2(448) - m'),
+# and 2^t by the documented exp2 algorithm below.  Everything else (the running
+# sum l, the rescale factors, PV and the output) stays in fp64.
+
+LOG2E_F32 = np.float32(1.4426950408889634)
+LOG2_448_F32 = np.float32(8.807354922057604)
+MAGIC_F32 = np.float32(12582912.0)           # 1.5 * 2^23
+EXP2_COEF_F32 = tuple(np.array([0x3F800000, 0x3F317AFE, 0x3E78062F, 0x3D6150BE],
+                               dtype=np.uint32).view(np.float32))
+
+
+def fma_f32(a, b, c) -> np.ndarray:
+    """fp32 fused multiply-add a*b + c with a single round-to-nearest-even.
+
+    a*b of two fp32 values is exact in fp64; TwoSum gives the fp64 sum s and
+    its exact error e; rounding s to fp32 is then correct unless s sits exactly
+    on an fp32 midpoint, where the sign of e decides the direction.
+    """
+    a = np.asarray(a, dtype=np.float32).astype(np.float64)
+    b = np.asarray(b, dtype=np.float32).astype(np.float64)
+    c = np.asarray(c, dtype=np.float32).astype(np.float64)
+    p = a * b
+    s = p + c
+    bb = s - p
+    e = (p - (s - bb)) + (c - bb)
+    r = s.astype(np.float32)
+    r64 = r.astype(np.float64)
+    up = np.nextafter(r, np.float32(np.inf))
+    dn = np.nextafter(r, np.float32(-np.inf))
+    # s exactly halfway between r and a neighbour: the exact sum s + e decides
+    tie_up = (s > r64) & (s - r64 == (up.astype(np.float64) - r64) / 2) & (e > 0)
+    tie_dn = (s < r64) & (r64 - s == (r64 - dn.astype(np.float64)) / 2) & (e < 0)
+    r = np.where(tie_up, up, np.where(tie_dn, dn, r))
+    return r.astype(np.float32)
+
+
+def exp2_f32(t) -> np.ndarray:
+    """2^t in fp32 operations: t clamped at -125, n = rint(t) by magic-number
+    rounding, f = t - n in [-1/2, 1/2], Horner polynomial 1 + c1 f + c2 f^2 + c3 f^3
+    (fp32 FMAs), and n added to the exponent field."""
+    t = np.maximum(np.asarray(t, dtype=np.float32), np.float32(-125.0))
+    r = (t + MAGIC_F32).astype(np.float32)
+    n = r.view(np.int32) - np.int32(0x4B400000)
+    f = (t - (r - MAGIC_F32).astype(np.float32)).astype(np.float32)
+    c0, c1, c2, c3 = EXP2_COEF_F32
+    p = fma_f32(c3, f, c2)
+    p = fma_f32(p, f, c1)
+    p = fma_f32(p, f, c0)
+    return (p.view(np.int32) + (n << 23)).view(np.float32)
+
+
+def kernel_scale_log2(d: int, sm_scale: float | None = None) -> np.float32:
+    """sm_scale * log2(e) as the kernel forms it in fp32 (default 1/sqrt(d))."""
+    s = (np.float32(1.0) / np.sqrt(np.float32(d))) if sm_scale is None else np.float32(sm_scale)
+    return np.float32(s * LOG2E_F32)
+
+
+def online_softmax_pv_fp32_decision(s_int, sq_rows, sk_blocks, scale_log2, valid, vvals, sv,
+                                    quantize_p: bool = True):
+    """Online softmax with the P8 codes decided in the kernel's fp32 precision.
+
+    s_int: (r, n_kv) exact scores; sq_rows: (r,) float32 Q scales; sk_blocks:
+    float32 K scales per 64-key block; scale_log2: float32 sm_scale*log2(e);
+    valid: (r, n_kv) bool key mask; vvals (n_kv, d) and sv (d,) as in
+    online_softmax_pv.  The running max m' is the fp32 max of fp32 products of
+    each 64-key half's largest score with that half's scale factor.
+    Returns (out, lse).
+    """
+    r, n_kv = s_int.shape
+    d = vvals.shape[1]
+    nblk = 2 * (-(-n_kv // KV_TILE))
+    skb = np.zeros(nblk, dtype=np.float32)
+    skb[:len(sk_blocks)] = sk_blocks
+    sq_rows = np.asarray(sq_rows, dtype=np.float32)
+    m32 = np.full(r, -np.inf, dtype=np.float32)
+    l = np.zeros(r)
+    o = np.zeros((r, d))
+    for j, t0 in enumerate(range(0, n_kv, KV_TILE)):
+        cols = np.arange(t0, min(n_kv, t0 + KV_TILE))
+        S = s_int[:, cols].astype(np.int64)
+        ok = valid[:, cols]
+        half = (cols - t0) // BLKK
+        ck = np.stack([((sq_rows * skb[2 * j + h]).astype(np.float32) * scale_log2).astype(np.float32)
+                       for h in (0, 1)], axis=1)                                   # (r, 2)
+        mt = np.full(r, -np.inf, dtype=np.float32)
+        for h in (0, 1):
+            sel = half == h
+            if not np.any(sel):
+                continue
+            Sh = np.where(ok[:, sel], S[:, sel], np.iinfo(np.int64).min)
+            imax = Sh.max(axis=1)
+            has = imax != np.iinfo(np.int64).min
+            prod = (imax.astype(np.float32) * ck[:, h]).astype(np.float32)
+            mt = np.maximum(mt, np.where(has, prod, np.float32(-np.inf)))
+        m_new = np.maximum(m32, mt)
+        nbias = (LOG2_448_F32 - m_new).astype(np.float32)
+        ckc = ck[:, half]                                                          # (r, T)
+        tt = fma_f32(S.astype(np.float32), ckc, nbias[:, None])
+        p = np.where(ok, exp2_f32(tt).astype(np.float64), 0.0)
+        p8 = e4m3_round(p) if quantize_p else p
+        # fp64 accumulation in the frame of the fp32 running max (log2 domain)
+        alpha = np.where(np.isfinite(m32), np.exp2(m32.astype(np.float64) - m_new.astype(np.float64)), 0.0)
+        x_log2 = S * (sq_rows.astype(np.float64)[:, None] * skb[2 * j + half].astype(np.float64)[None, :]) \
+            * float(scale_log2)
+        e = np.where(ok, P_SCALE * np.exp2(x_log2 - m_new.astype(np.float64)[:, None]), 0.0)
+        l = l * alpha + np.sum(e, axis=1)
+        o = o * alpha[:, None] + p8 @ vvals[cols]
+        m32 = m_new
+    out = o * sv[None, :] / l[:, None]
+    lse = m32.astype(np.float64) * math.log(2.0) + np.log(l / P_SCALE)
+    return out, lse
+
+
+def attention_head_kernel_precision(q, k, v, *, causal=False, sm_scale=None, rows=None,
+                                    quantize_p: bool = True) -> dict:
+    """attention_head with the P8 codes decided in the kernel's fp32 precision.
+
+    Quantization of Q, K, V and the integer scores are the same exact stages as
+    attention_head; l, the rescale factors, PV and the output are fp64.
+    """
+    q = np.asarray(q, dtype=np.float32)
+    k = np.asarray(k, dtype=np.float32)
+    v = np.asarray(v, dtype=np.float32)
+    n, d = q.shape
+    n_kv = k.shape[0]
+    if causal and n != n_kv:
+        raise ValueError("causal attention needs equal query and key lengths")
+    rows = np.arange(n) if rows is None else np.asarray(rows, dtype=np.int64)
+    mu = k_channel_mean(k)
+    q8, sq = quantize_int8_blocks(q, BLKQ)
+    k8, sk = quantize_int8_blocks(smooth_k(k, mu), BLKK)
+    v8, sv = quantize_v_e4m3(v)
+    s_int = integer_scores(q8[rows], k8[:n_kv])
+    valid = np.ones((len(rows), n_kv), dtype=bool)
+    if causal:
+        valid = np.arange(n_kv)[None, :] <= rows[:, None]
+    out, lse = online_softmax_pv_fp32_decision(
+        s_int, sq[rows // BLKQ], sk, kernel_scale_log2(d, sm_scale), valid,
+        e4m3_decode(v8), sv.astype(np.float64), quantize_p=quantize_p)
+    return dict(out=out, lse=lse, rows=rows, k_mean=mu, q8=q8, q_scale=sq, k8=k8, k_scale=sk,
+                v8=v8, v_scale=sv, s_int=s_int)

@@ -26,7 +26,7 @@
 // Per KV tile j the softmax thread of query row i (log2 domain, u = x * log2 e):
 //   u_j   = S_ij * (q_scale * k_scale_j * sm_scale * log2 e)
 //   m'    = max(m, max_j u_j);  alpha = 2^(m - m')
-//   p_j   = 2^(u_j - m' + log2 448)   (= 448 * exp(x_j - x_max'))
+//   p_j   = 2^(u_j - m' + log2 448)   (= 448 * exp(x_j - x_max'), exp2_poly below)
 //   l     = l * alpha + sum_j p_j     (unquantized), P8_j = e4m3(p_j) -> TMEM
 //   O     = O * alpha + PV_blk        (PV_blk = P8 V8 in FP32, fresh each tile)
 //   out   = O * v_scale / l ;  lse = m' ln 2 + ln(l / 448)
@@ -82,13 +82,33 @@ struct AttnSmem {
 
 __device__ __forceinline__ float i2f_exact(uint32_t s) {
   // exact int32 -> fp32 for |s| < 2^22: place s in the mantissa of 1.5 * 2^23
-  return __int_as_float(static_cast<int>(s) + 0x4B400000) - 12582912.0f;
+  return __fsub_rn(__int_as_float(static_cast<int>(s) + 0x4B400000), 12582912.0f);
 }
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^t in plain IEEE fp32 operations, so that the P8 code it decides can be
+// reproduced exactly on any host: Cody-Waite split t = n + f with n = rint(t)
+// (magic-number rounding) and f in [-1/2, 1/2], a degree-3 polynomial for 2^f
+// (coefficients fitted for minimal relative error with the constant term fixed
+// at 1; max relative error 1.0e-4), and n added to the exponent field.  t is
+// clamped at -125 so the result stays a normal number.
+constexpr float kExp2C1 = 0.693282962f;   // 0x3f317afe
+constexpr float kExp2C2 = 0.242211089f;   // 0x3e78062f
+constexpr float kExp2C3 = 0.0550086424f;  // 0x3d6150be
+__device__ __forceinline__ float exp2_poly(float t) {
+  t = fmaxf(t, -125.0f);
+  const float r = __fadd_rn(t, 12582912.0f);
+  const int n = __float_as_int(r) - 0x4B400000;
+  const float f = __fsub_rn(t, __fsub_rn(r, 12582912.0f));
+  float p = __fmaf_rn(kExp2C3, f, kExp2C2);
+  p = __fmaf_rn(p, f, kExp2C1);
+  p = __fmaf_rn(p, f, 1.0f);
+  return __int_as_float(__float_as_int(p) + (n << 23));
 }
 
 template <int D, class Seq>
@@ -316,8 +336,8 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kBlkK) + off / kBlkK;
 
     for (int j = 0; j < nkv[t] && ok; ++j) {
-      const float ck0 = sq * ksc[2 * j] * a.scale_log2;
-      const float ck1 = sq * ksc[2 * j + 1] * a.scale_log2;
+      const float ck0 = __fmul_rn(__fmul_rn(sq, ksc[2 * j]), a.scale_log2);
+      const float ck1 = __fmul_rn(__fmul_rn(sq, ksc[2 * j + 1]), a.scale_log2);
       const bool masked = (a.causal && j == qt[t]) || (j + 1) * kKvTile > n;
       const int kv0 = j * kKvTile;
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s(t), j & 1, 0x301 + t));
@@ -345,11 +365,11 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         }
         if (c < 2) imax0 = max(imax0, mx); else imax1 = max(imax1, mx);
       }
-      const float mt = fmaxf(imax0 == INT_MIN ? -INFINITY : static_cast<float>(imax0) * ck0,
-                             imax1 == INT_MIN ? -INFINITY : static_cast<float>(imax1) * ck1);
+      const float mt = fmaxf(imax0 == INT_MIN ? -INFINITY : __fmul_rn(static_cast<float>(imax0), ck0),
+                             imax1 == INT_MIN ? -INFINITY : __fmul_rn(static_cast<float>(imax1), ck1));
       const float m_new = fmaxf(m, mt);
       const float alpha = ex2(m - m_new);
-      const float nbias = kLog2_448 - m_new;
+      const float nbias = __fsub_rn(kLog2_448, m_new);
 
       // pass 2: p = 448 * 2^(u - m'), running sum, e4m3 P8 into TMEM over the S columns
       float lt = 0.0f;
@@ -365,7 +385,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
           float p[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            p[e] = ex2(fmaf(i2f_exact(r[4 * i + e]), ck, nbias));
+            p[e] = exp2_poly(__fmaf_rn(i2f_exact(r[4 * i + e]), ck, nbias));
             if (masked) {
               const int key = kv0 + 32 * c + 4 * i + e;
               if (key >= n || (a.causal && key > grow)) p[e] = 0.0f;

@@ -15,6 +15,10 @@ TORCH_DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
 MAX_ABS = 2e-3
 MIN_COS = 0.9999
 
+# (case, max-abs, cos) of every comparison; written out by conftest when
+# SAGE_PARITY_REPORT names a file
+REPORT = []
+
 
 def to_device(x: np.ndarray, dtype: str, layout: str, varlen: bool) -> torch.Tensor:
     t = torch.from_numpy(np.ascontiguousarray(x)).to(TORCH_DT[dtype])

@@ -368,3 +368,99 @@ def test_oracle_matches_its_committed_snapshot():
             assert hw[key] == hg[key], key
         assert np.max(np.abs(np.array(hw["out_rows"]) - np.array(hg["out_rows"]))) <= 1e-12
         assert np.max(np.abs(np.array(hw["lse_rows"]) - np.array(hg["lse_rows"]))) <= 1e-12
+
+
+# ---------------------------------------------------------------- kernel-precision P8 decision
+
+def _rn32_exact(fr):
+    """Round a Fraction to fp32, ties to even, by comparing exact distances."""
+    from fractions import Fraction
+    x = np.float32(float(fr))
+    best = None
+    for cand in (np.nextafter(x, np.float32(-np.inf)), x, np.nextafter(x, np.float32(np.inf))):
+        key = (abs(Fraction(float(cand)) - fr), int(np.float32(cand).view(np.uint32)) & 1)
+        if best is None or key < best[0]:
+            best = (key, cand)
+    return np.float32(best[1])
+
+
+def test_fma_f32_is_a_single_rounding():
+    from fractions import Fraction
+    rng = np.random.default_rng(21)
+    n = 4000
+    a, b, c = ((rng.standard_normal(n) * 10.0 ** rng.uniform(-6, 6, n)).astype(np.float32)
+               for _ in range(3))
+    got = orc.fma_f32(a, b, c)
+    for i in range(n):
+        want = _rn32_exact(Fraction(float(a[i])) * Fraction(float(b[i])) + Fraction(float(c[i])))
+        assert got[i] == want, i
+    # exact midpoints of the fp64 sum: the discarded error must decide the direction
+    a2 = np.float32([2 ** -12, 2 ** -12, 1 + 2 ** -23, 3.0])
+    b2 = np.float32([2 ** -12 * (1 + 2 ** -23), 2 ** -12 * (1 - 2 ** -24), 2 ** -24, 2 ** -25])
+    c2 = np.float32([1, 1, 1, 1])
+    for x, p, q, w in zip(orc.fma_f32(a2, b2, c2), a2, b2, c2):
+        assert x == _rn32_exact(Fraction(float(p)) * Fraction(float(q)) + Fraction(float(w)))
+
+
+def test_exp2_f32_accuracy_and_exact_powers():
+    t = np.linspace(-125, 9, 400001).astype(np.float32)
+    p = orc.exp2_f32(t).astype(np.float64)
+    assert np.max(np.abs(p / np.exp2(t.astype(np.float64)) - 1)) <= 1.02e-4
+    ti = np.arange(-125, 10).astype(np.float32)
+    assert np.array_equal(orc.exp2_f32(ti), np.exp2(ti))
+    assert np.all(np.diff(orc.exp2_f32(np.linspace(-3, 3, 10001).astype(np.float32))) >= 0)
+    assert orc.exp2_f32(np.float32([-1000.0]))[0] == np.float32(2.0 ** -125)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_kernel_precision_path_without_p_rounding_is_softmax_attention(causal):
+    # with P left unrounded, the only approximation is the exp2 polynomial (1e-4)
+    rng = np.random.default_rng(22)
+    n, d = 333, 64
+    q, k, v = (rng.standard_normal((n, d)).astype(np.float32) for _ in range(3))
+    a = orc.attention_head_kernel_precision(q, k, v, causal=causal, quantize_p=False)
+    r = orc.attention_head(q, k, v, causal=causal, quantize=True)
+    # same quantized logits and V; compare against the fp64 path with P unrounded
+    x = r["s_int"].astype(np.float64) * r["q_scale"][np.arange(n) // orc.BLKQ, None] \
+        * r["k_scale"][None, np.arange(n) // orc.BLKK] / math.sqrt(d)
+    if causal:
+        x = np.where(np.arange(n)[None, :] > np.arange(n)[:, None], -np.inf, x)
+    ref, lse = orc.online_softmax_pv(x, orc.e4m3_decode(r["v8"]), r["v_scale"].astype(np.float64),
+                                     quantize_p=False)
+    scale = np.max(np.abs(ref))
+    assert np.max(np.abs(a["out"] - ref)) <= 3e-4 * scale
+    assert np.max(np.abs(a["lse"] - lse)) <= 1e-5
+
+
+def test_kernel_precision_decision_matches_fp64_definition_closely():
+    w = WORKLOADS["tiny"]
+    x = generate(w)
+    for h in range(2):
+        a = orc.attention_head_kernel_precision(x["q"][0, h], x["k"][0, h], x["v"][0, h])
+        b = orc.attention_head(x["q"][0, h], x["k"][0, h], x["v"][0, h])
+        err = np.max(np.abs(a["out"] - b["out"]))
+        cos = float(a["out"].ravel() @ b["out"].ravel() /
+                    (np.linalg.norm(a["out"]) * np.linalg.norm(b["out"])))
+        assert cos >= 0.9999 and err <= 5e-3
+        assert np.max(np.abs(a["lse"] - b["lse"])) <= 1e-5
+
+
+def test_kernel_precision_p8_codes_mostly_equal_fp64_codes():
+    rng = np.random.default_rng(23)
+    n, d = 256, 128
+    q, k, v = (rng.standard_normal((n, d)).astype(np.float32) for _ in range(3))
+    r = orc.attention_head(q, k, v)
+    sc = orc.kernel_scale_log2(d)
+    s = r["s_int"][:, :128].astype(np.int64)
+    ck = (r["q_scale"][0] * r["k_scale"][np.arange(128) // 64]).astype(np.float32) * sc
+    ck = ck.astype(np.float32)
+    u = (s.astype(np.float32) * ck[None, :]).astype(np.float32)
+    # one tile, first block: both definitions start from the same row max
+    m = np.maximum((s[:, :64].max(1).astype(np.float32) * ck[0]).astype(np.float32),
+                   (s[:, 64:].max(1).astype(np.float32) * ck[64]).astype(np.float32))
+    t = orc.fma_f32(s.astype(np.float32), ck[None, :], (orc.LOG2_448_F32 - m)[:, None])
+    p32 = orc.e4m3_round(orc.exp2_f32(t).astype(np.float64))
+    x = s * ck[None, :].astype(np.float64)
+    p64 = orc.e4m3_round(448.0 * np.exp2(x - x.max(1, keepdims=True)))
+    assert np.mean(p32 == p64) >= 0.995
+    del u
