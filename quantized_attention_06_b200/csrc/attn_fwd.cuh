@@ -111,6 +111,105 @@ __device__ __forceinline__ float exp2_poly(float t) {
   return __int_as_float(__float_as_int(p) + (n << 23));
 }
 
+// ---- packed fp32 pair arithmetic (one instruction per two values)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(reinterpret_cast<uint64_t&>(d))
+      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)),
+        "l"(reinterpret_cast<const uint64_t&>(c)));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(reinterpret_cast<uint64_t&>(d))
+      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Wait for this thread's TMEM loads; tying the destination registers keeps the
+// compiler from using them before the wait.
+__device__ __forceinline__ void tmem_wait_ld_tied(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld_tied(uint32_t (&a)[32], uint32_t (&b)[32]) {
+  tmem_wait_ld_tied(a);
+  asm volatile(""
+               : "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]),
+                 "+r"(b[6]), "+r"(b[7]), "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]),
+                 "+r"(b[12]), "+r"(b[13]), "+r"(b[14]), "+r"(b[15]), "+r"(b[16]), "+r"(b[17]),
+                 "+r"(b[18]), "+r"(b[19]), "+r"(b[20]), "+r"(b[21]), "+r"(b[22]), "+r"(b[23]),
+                 "+r"(b[24]), "+r"(b[25]), "+r"(b[26]), "+r"(b[27]), "+r"(b[28]), "+r"(b[29]),
+                 "+r"(b[30]), "+r"(b[31])
+               :
+               : "memory");
+}
+
+// Largest non-negative score among 32 int32 values read as fp32 bit patterns:
+// non-negative scores are ordered subnormals, negative ones are NaN, which max
+// ignores.  Returns NaN when no score is non-negative.
+__device__ __forceinline__ float max_nonneg32(const uint32_t (&r)[32], float acc) {
+  float m0 = acc, m1 = __uint_as_float(0xFFFFFFFFu), m2 = m1, m3 = m1;
+#pragma unroll
+  for (int i = 0; i < 32; i += 8) {
+    m0 = fmax3(m0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+    m1 = fmax3(m1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+    m2 = fmax3(m2, __uint_as_float(r[i + 4]), __uint_as_float(r[i + 5]));
+    m3 = fmax3(m3, __uint_as_float(r[i + 6]), __uint_as_float(r[i + 7]));
+  }
+  return fmax3(m0, m1, fmaxf(m2, m3));
+}
+
+// P for 32 keys of one 64-key half: t = fma(12582912 + S, ck, cb) with
+// cb = (log2 448 - m') - 12582912 * ck, p = exp2_poly(t); returns e4m3 codes
+// packed four per word and adds p into acc.  The same fp32 operations as
+// exp2_poly, two values per instruction.
+__device__ __forceinline__ void p8_chunk(const uint32_t (&r)[32], float ck, float cb, float2& acc,
+                                         uint32_t (&w)[8]) {
+  const float2 CK = make_float2(ck, ck), CB = make_float2(cb, cb);
+  const float2 M = make_float2(12582912.0f, 12582912.0f), NM = make_float2(-12582912.0f, -12582912.0f);
+  const float2 NEG1 = make_float2(-1.0f, -1.0f), ONE = make_float2(1.0f, 1.0f);
+  const float2 C1 = make_float2(kExp2C1, kExp2C1), C2 = make_float2(kExp2C2, kExp2C2);
+  const float2 C3 = make_float2(kExp2C3, kExp2C3);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float2 pp[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int e = 4 * i + 2 * h;
+      const float2 x = make_float2(__int_as_float(static_cast<int>(r[e]) + 0x4B400000),
+                                   __int_as_float(static_cast<int>(r[e + 1]) + 0x4B400000));
+      float2 t = ffma2(x, CK, CB);
+      t.x = fmaxf(t.x, -125.0f);
+      t.y = fmaxf(t.y, -125.0f);
+      const float2 rr = fadd2(t, M);
+      const float2 f = ffma2(fadd2(rr, NM), NEG1, t);
+      float2 p = ffma2(C3, f, C2);
+      p = ffma2(p, f, C1);
+      p = ffma2(p, f, ONE);
+      p.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(rr.x) << 23));
+      p.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(rr.y) << 23));
+      pp[h] = p;
+    }
+    acc = fadd2(acc, fadd2(pp[0], pp[1]));
+    w[i] = e4m3x2(pp[0].x, pp[0].y) | (e4m3x2(pp[1].x, pp[1].y) << 16);
+  }
+}
+
 template <int D, class Seq>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
@@ -325,9 +424,9 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const uint32_t tS = tmem + lane_base + kColS0 + 128u * t;
     const uint32_t tPV = tmem + lane_base + kColPV0 + 128u * t;
 
-    float o[D];
+    float2 o2[D / 2];
 #pragma unroll
-    for (int c = 0; c < D; ++c) o[c] = 0.0f;
+    for (int c = 0; c < D / 2; ++c) o2[c] = make_float2(0.0f, 0.0f);
     float m = -INFINITY, l = 0.0f;
     bool ok = !dead;
     const float sq = (nkv[t] > 0) ? a.q_scale[static_cast<int64_t>(hq) * (seq.t_pad / kBlkQ) +
@@ -344,76 +443,139 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       if (!ok) break;
       tc_fence_after();
 
-      // pass 1: row maximum of the integer scores in each 64-key half
-      int imax0 = INT_MIN, imax1 = INT_MIN;
+      // masked keys (past the sequence end or above the causal diagonal) read as NaN
+      auto mask_chunk = [&](uint32_t (&r)[32], int c) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + 32u * c, r);
-        tmem_wait_ld();
-        int mx = INT_MIN;
-        if (masked) {
+        for (int i = 0; i < 32; ++i) {
+          const int key = kv0 + 32 * c + i;
+          if (key >= n || (a.causal && key > grow)) r[i] = 0xFFFFFFFFu;
+        }
+      };
+
+      // pass 1: largest score of each 64-key half
+      float hmax[2];
+      {
+        uint32_t ra[32], rb[32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          tmem_ld32(tS + 64u * h, ra);
+          tmem_ld32(tS + 64u * h + 32u, rb);
+          tmem_wait_ld_tied(ra, rb);
+          if (masked) { mask_chunk(ra, 2 * h); mask_chunk(rb, 2 * h + 1); }
+          hmax[h] = max_nonneg32(rb, max_nonneg32(ra, __uint_as_float(0xFFFFFFFFu)));
+        }
+      }
+      int imax[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        imax[h] = static_cast<int>(__float_as_uint(hmax[h]));
+        if (isnan(hmax[h])) {  // no non-negative score in this half: exact integer max
+          uint32_t ra[32], rb[32];
+          tmem_ld32(tS + 64u * h, ra);
+          tmem_ld32(tS + 64u * h + 32u, rb);
+          tmem_wait_ld_tied(ra, rb);
+          int mx = INT_MIN;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const int key = kv0 + 32 * c + i;
-            const bool drop = key >= n || (a.causal && key > grow);
-            mx = max(mx, drop ? INT_MIN : static_cast<int>(r[i]));
+            const int k0 = kv0 + 64 * h + i, k1 = k0 + 32;
+            const bool d0 = masked && (k0 >= n || (a.causal && k0 > grow));
+            const bool d1 = masked && (k1 >= n || (a.causal && k1 > grow));
+            mx = d0 ? mx : max(mx, static_cast<int>(ra[i]));
+            mx = d1 ? mx : max(mx, static_cast<int>(rb[i]));
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mx = max(mx, static_cast<int>(r[i]));
+          imax[h] = mx;
         }
-        if (c < 2) imax0 = max(imax0, mx); else imax1 = max(imax1, mx);
       }
-      const float mt = fmaxf(imax0 == INT_MIN ? -INFINITY : __fmul_rn(static_cast<float>(imax0), ck0),
-                             imax1 == INT_MIN ? -INFINITY : __fmul_rn(static_cast<float>(imax1), ck1));
+      const float mt = fmaxf(imax[0] == INT_MIN ? -INFINITY : __fmul_rn(static_cast<float>(imax[0]), ck0),
+                             imax[1] == INT_MIN ? -INFINITY : __fmul_rn(static_cast<float>(imax[1]), ck1));
       const float m_new = fmaxf(m, mt);
       const float alpha = ex2(m - m_new);
       const float nbias = __fsub_rn(kLog2_448, m_new);
+      const float cb0 = __fsub_rn(nbias, __fmul_rn(12582912.0f, ck0));
+      const float cb1 = __fsub_rn(nbias, __fmul_rn(12582912.0f, ck1));
 
       // pass 2: p = 448 * 2^(u - m'), running sum, e4m3 P8 into TMEM over the S columns
-      float lt = 0.0f;
+      float2 acc = make_float2(0.0f, 0.0f);
+      {
+        uint32_t ra[32], rb[32], w[8];
+        auto finish = [&](uint32_t (&r)[32], int c) {
+          if (masked) {
+            float2 dummy = make_float2(0.0f, 0.0f);
+            p8_chunk(r, c < 2 ? ck0 : ck1, c < 2 ? cb0 : cb1, dummy, w);
+            // recompute with masked entries zeroed (tiles on the diagonal / sequence tail)
+            float2 acc_m = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + 32u * c, r);
-        tmem_wait_ld();
-        const float ck = (c < 2) ? ck0 : ck1;
-        uint32_t w[8];
+            for (int i = 0; i < 8; ++i) {
+              uint32_t code = w[i];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float p[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            p[e] = exp2_poly(__fmaf_rn(i2f_exact(r[4 * i + e]), ck, nbias));
-            if (masked) {
-              const int key = kv0 + 32 * c + 4 * i + e;
-              if (key >= n || (a.causal && key > grow)) p[e] = 0.0f;
+              for (int e = 0; e < 4; ++e) {
+                const int key = kv0 + 32 * c + 4 * i + e;
+                if (key >= n || (a.causal && key > grow)) code &= ~(0xFFu << (8 * e));
+              }
+              w[i] = code;
             }
+            // the running sum needs the unquantized values of the kept keys only
+            {
+              const float ck = c < 2 ? ck0 : ck1, cb = c < 2 ? cb0 : cb1;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int key = kv0 + 32 * c + i;
+                const float tt = __fmaf_rn(__int_as_float(static_cast<int>(r[i]) + 0x4B400000), ck, cb);
+                const float pv = exp2_poly(tt);
+                if (!(key >= n || (a.causal && key > grow))) acc_m.x = __fadd_rn(acc_m.x, pv);
+              }
+            }
+            acc = fadd2(acc, acc_m);
+            (void)dummy;
+          } else {
+            p8_chunk(r, c < 2 ? ck0 : ck1, c < 2 ? cb0 : cb1, acc, w);
           }
-          lt += (p[0] + p[1]) + (p[2] + p[3]);
-          w[i] = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
-        }
-        tmem_st8(tS + 8u * c, w);
+          tmem_st8(tS + 8u * c, w);
+        };
+        tmem_ld32(tS, ra);
+        tmem_wait_ld_tied(ra);
+        tmem_ld32(tS + 32u, rb);
+        finish(ra, 0);
+        tmem_wait_ld_tied(rb);
+        tmem_ld32(tS + 64u, ra);
+        finish(rb, 1);
+        tmem_wait_ld_tied(ra);
+        tmem_ld32(tS + 96u, rb);
+        finish(ra, 2);
+        tmem_wait_ld_tied(rb);
+        finish(rb, 3);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_p(t));
-      l = l * alpha + lt;
+      l = l * alpha + (acc.x + acc.y);
       m = m_new;
 
       // two-level accumulation: O = alpha * O + PV_blk (PV_blk fresh in TMEM for this tile)
       ok = __all_sync(0xffffffffu, mbar_wait(bar_pv(t), j & 1, 0x303 + t));
       if (!ok) break;
       tc_fence_after();
+      {
+        const float2 al = make_float2(alpha, alpha);
+        uint32_t ra[32], rb[32];
+        auto accum = [&](const uint32_t (&r)[32], int c) {
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tPV + 32u * c, r);
-        tmem_wait_ld();
+          for (int i = 0; i < 16; ++i)
+            o2[16 * c + i] = ffma2(o2[16 * c + i], al,
+                                   make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])));
+        };
+        tmem_ld32(tPV, ra);
+        tmem_wait_ld_tied(ra);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[32 * c + i] = fmaf(o[32 * c + i], alpha, __uint_as_float(r[i]));
+        for (int c = 0; c < D / 32; c += 2) {
+          tmem_ld32(tPV + 32u * (c + 1), rb);
+          accum(ra, c);
+          tmem_wait_ld_tied(rb);
+          if (c + 2 < D / 32) tmem_ld32(tPV + 32u * (c + 2), ra);
+          accum(rb, c + 1);
+          if (c + 2 < D / 32) tmem_wait_ld_tied(ra);
+        }
       }
     }
 
@@ -426,8 +588,8 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         float* dst = reinterpret_cast<float*>(a.out) + orow;
 #pragma unroll
         for (int c = 0; c < D; c += 4) {
-          float4 v = make_float4(o[c] * vs[c] * inv_l, o[c + 1] * vs[c + 1] * inv_l,
-                                 o[c + 2] * vs[c + 2] * inv_l, o[c + 3] * vs[c + 3] * inv_l);
+          float4 v = make_float4(o2[c / 2].x * vs[c] * inv_l, o2[c / 2].y * vs[c + 1] * inv_l,
+                                 o2[c / 2 + 1].x * vs[c + 2] * inv_l, o2[c / 2 + 1].y * vs[c + 3] * inv_l);
           *reinterpret_cast<float4*>(dst + c) = v;
         }
       } else if (a.out_dtype == 1) {
@@ -436,7 +598,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         for (int c = 0; c < D; c += 8) {
           __align__(16) __nv_bfloat16 h8[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) h8[i] = __float2bfloat16_rn(o[c + i] * vs[c + i] * inv_l);
+          for (int i = 0; i < 8; ++i) h8[i] = __float2bfloat16_rn(((i & 1) ? o2[(c + i) / 2].y : o2[(c + i) / 2].x) * vs[c + i] * inv_l);
           *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<const uint4*>(h8);
         }
       } else {
@@ -445,7 +607,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         for (int c = 0; c < D; c += 8) {
           __align__(16) __half h8[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) h8[i] = __float2half_rn(o[c + i] * vs[c + i] * inv_l);
+          for (int i = 0; i < 8; ++i) h8[i] = __float2half_rn(((i & 1) ? o2[(c + i) / 2].y : o2[(c + i) / 2].x) * vs[c + i] * inv_l);
           *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<const uint4*>(h8);
         }
       }

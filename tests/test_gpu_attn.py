@@ -63,7 +63,9 @@ def _check(x, w, causal, pairs, out_dtype=torch.float32):
             assert mx <= MAX_ABS, (b, h, mx)
         else:
             o_ref_r = torch.from_numpy(o_ref).to(out_dtype).double().numpy()
-            ulp = np.abs(o_ref_r) * (2.0 ** -8 if out_dtype == torch.bfloat16 else 2.0 ** -11)
+            mant = 7 if out_dtype == torch.bfloat16 else 10        # explicit mantissa bits
+            _, ex = np.frexp(np.maximum(np.abs(o_ref_r), 2.0 ** -14))
+            ulp = np.ldexp(1.0, ex - 1 - mant)                      # one unit in the last place
             assert np.all(np.abs(o_gpu - o_ref_r) <= MAX_ABS + ulp), (b, h)
             _, cos, _ = metrics(o_gpu, o_ref)
         REPORT.append({"case": f"{w.name} causal={causal} out={out_dtype} b={b} h={h}",
