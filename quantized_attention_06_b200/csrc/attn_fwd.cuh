@@ -469,7 +469,9 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         imax[h] = static_cast<int>(__float_as_uint(hmax[h]));
-        if (isnan(hmax[h])) {  // no non-negative score in this half: exact integer max
+        // a row with no non-negative score in this half needs the exact integer max; the
+        // TMEM reload is warp-collective, so the whole warp takes this branch together
+        if (__any_sync(0xffffffffu, isnan(hmax[h]))) {
           uint32_t ra[32], rb[32];
           tmem_ld32(tS + 64u * h, ra);
           tmem_ld32(tS + 64u * h + 32u, rb);
@@ -483,7 +485,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mx = d0 ? mx : max(mx, static_cast<int>(ra[i]));
             mx = d1 ? mx : max(mx, static_cast<int>(rb[i]));
           }
-          imax[h] = mx;
+          if (isnan(hmax[h])) imax[h] = mx;
         }
       }
       const float mt = fmaxf(imax[0] == INT_MIN ? -INFINITY : __fmul_rn(static_cast<float>(imax[0]), ck0),
