@@ -22,7 +22,7 @@ What it computes, stage by stage, for one (sequence, query head) with its KV hea
 Everything after the integer scores is done in float64, with one exception
 kept apart in ``attention_head_kernel_precision``: P8 is an integer code decided
 by floating point, so for GPU parity that decision is taken with the kernel's
-own fp32 steps (fp32 logits and running max, t = fma(12582912 + S, ck, cb),
+own fp32 steps (fp32 logits and running max, t = fma(S, ck, log2 448 - m'),
 the documented fp32 exp2 algorithm, e4m3 rounding); l, the rescale factors, PV
 and the output stay fp64.  ``attention_head`` is the all-fp64 definition.
 
@@ -345,9 +345,8 @@ def reference_attention(q, k, v, *, causal=False, sm_scale=None) -> np.ndarray:
 # --------------------------------------------------------------------------
 # P8 is an integer code decided by floating point, so for parity both sides take
 # that decision with the same fp32 arithmetic: logits u = S * ck in the log2
-# domain, the running max m' over 64-key halves, t = fma(12582912 + S, ck, cb)
-# with cb = fp32(fp32(log2 448 - m') - fp32(12582912 * ck)), and 2^t by the
-# documented exp2 algorithm below.  Everything else (the running
+# domain, the running max m' over 64-key halves, t = fma(S, ck, log2(448) - m'),
+# and 2^t by the documented exp2 algorithm below.  Everything else (the running
 # sum l, the rescale factors, PV and the output) stays in fp64.
 
 LOG2E_F32 = np.float32(1.4426950408889634)
@@ -442,12 +441,8 @@ def online_softmax_pv_fp32_decision(s_int, sq_rows, sk_blocks, scale_log2, valid
             mt = np.maximum(mt, np.where(has, prod, np.float32(-np.inf)))
         m_new = np.maximum(m32, mt)
         nbias = (LOG2_448_F32 - m_new).astype(np.float32)
-        # t = fma(12582912 + S, ck, cb), cb = (log2 448 - m') - 12582912 * ck: the
-        # int32 -> fp32 conversion offset of the kernel folded into the bias
-        cb = (nbias[:, None] - (MAGIC_F32 * ck).astype(np.float32)).astype(np.float32)  # (r, 2)
         ckc = ck[:, half]                                                          # (r, T)
-        cbc = cb[:, half]
-        tt = fma_f32((S + 12582912).astype(np.float32), ckc, cbc)
+        tt = fma_f32(S.astype(np.float32), ckc, nbias[:, None])
         p = np.where(ok, exp2_f32(tt).astype(np.float64), 0.0)
         p8 = e4m3_round(p) if quantize_p else p
         # fp64 accumulation in the frame of the fp32 running max (log2 domain)

@@ -24,7 +24,7 @@
 // MMA that reads them, and tcgen05.mma ops of one thread execute in issue order.
 //
 // Per KV tile j the softmax thread of query row i (log2 domain, u = x * log2 e):
-//   u_j   = S_ij * (q_scale * k_scale_j * sm_scale * log2 e)
+//   u_j   = S_ij * (q_scale * k_scale_j * sm_scale * log2 e)   (S read as 12582912 + S)
 //   m'    = max(m, max_j u_j);  alpha = 2^(m - m')
 //   p_j   = 2^(u_j - m' + log2 448)   (= 448 * exp(x_j - x_max'), exp2_poly below)
 //   l     = l * alpha + sum_j p_j     (unquantized), P8_j = e4m3(p_j) -> TMEM
@@ -73,8 +73,8 @@ struct AttnSmem {
   static constexpr int kVOff = kKOff + kKStages * kTileQ;
   static constexpr int kBarOff = kVOff + kVStages * kTileV;
   // barriers: q_full, k_full[3], k_empty[3], v_full[3], v_empty[3], s_full[2], p_full[2],
-  // pv_full[2], mma_done  -> 20 x 8 bytes, then the TMEM address slot
-  static constexpr int kNumBars = 20;
+  // pv_full[2], mma_done, s_free[2]  -> 22 x 8 bytes, then the TMEM address slot
+  static constexpr int kNumBars = 22;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kSlotOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
@@ -159,11 +159,27 @@ __device__ __forceinline__ void tmem_wait_ld_tied(uint32_t (&a)[32], uint32_t (&
                : "memory");
 }
 
-// Largest non-negative score among 32 int32 values read as fp32 bit patterns:
-// non-negative scores are ordered subnormals, negative ones are NaN, which max
-// ignores.  Returns NaN when no score is non-negative.
-__device__ __forceinline__ float max_nonneg32(const uint32_t (&r)[32], float acc) {
-  float m0 = acc, m1 = __uint_as_float(0xFFFFFFFFu), m2 = m1, m3 = m1;
+// The S region is pre-filled with kMagicBits (the fp32 1.5 * 2^23 = 12582912) and the
+// INT8 MMAs accumulate onto it, so TMEM returns bits(12582912 + S): an fp32 whose
+// value is exactly 12582912 + S for |S| < 2^22 (|S| <= d * 127^2 here).  Those values
+// are positive and ordered like S, and S itself is one exact subtraction away.
+constexpr uint32_t kMagicBits = 0x4B400000u;
+constexpr float kMagic = 12582912.0f;
+
+// 32 lanes x 32 consecutive columns of TMEM all set to kMagicBits.
+__device__ __forceinline__ void tmem_fill_magic32(uint32_t taddr) {
+  const uint32_t v = kMagicBits;
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
+      "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
+
+// max over 32 magic-offset scores (masked entries hold 0, below every valid value)
+__device__ __forceinline__ float max32(const uint32_t (&r)[32], float acc) {
+  float m0 = acc, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
 #pragma unroll
   for (int i = 0; i < 32; i += 8) {
     m0 = fmax3(m0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
@@ -174,14 +190,14 @@ __device__ __forceinline__ float max_nonneg32(const uint32_t (&r)[32], float acc
   return fmax3(m0, m1, fmaxf(m2, m3));
 }
 
-// P for 32 keys of one 64-key half: t = fma(12582912 + S, ck, cb) with
-// cb = (log2 448 - m') - 12582912 * ck, p = exp2_poly(t); returns e4m3 codes
-// packed four per word and adds p into acc.  The same fp32 operations as
-// exp2_poly, two values per instruction.
-__device__ __forceinline__ void p8_chunk(const uint32_t (&r)[32], float ck, float cb, float2& acc,
+// P for 32 keys of one 64-key half: S = (12582912 + S) - 12582912 (exact),
+// t = fma(S, ck, log2 448 - m'), p = exp2_poly(t) evaluated two values per
+// instruction (the same fp32 operations as exp2_poly).  Returns the e4m3 codes
+// packed four per word and adds p into acc.
+__device__ __forceinline__ void p8_chunk(const uint32_t (&r)[32], float ck, float nb, float2& acc,
                                          uint32_t (&w)[8]) {
-  const float2 CK = make_float2(ck, ck), CB = make_float2(cb, cb);
-  const float2 M = make_float2(12582912.0f, 12582912.0f), NM = make_float2(-12582912.0f, -12582912.0f);
+  const float2 CK = make_float2(ck, ck), NB = make_float2(nb, nb);
+  const float2 M = make_float2(kMagic, kMagic), NM = make_float2(-kMagic, -kMagic);
   const float2 NEG1 = make_float2(-1.0f, -1.0f), ONE = make_float2(1.0f, 1.0f);
   const float2 C1 = make_float2(kExp2C1, kExp2C1), C2 = make_float2(kExp2C2, kExp2C2);
   const float2 C3 = make_float2(kExp2C3, kExp2C3);
@@ -191,9 +207,8 @@ __device__ __forceinline__ void p8_chunk(const uint32_t (&r)[32], float ck, floa
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int e = 4 * i + 2 * h;
-      const float2 x = make_float2(__int_as_float(static_cast<int>(r[e]) + 0x4B400000),
-                                   __int_as_float(static_cast<int>(r[e + 1]) + 0x4B400000));
-      float2 t = ffma2(x, CK, CB);
+      const float2 x = fadd2(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), NM);
+      float2 t = ffma2(x, CK, NB);
       t.x = fmaxf(t.x, -125.0f);
       t.y = fmaxf(t.y, -125.0f);
       const float2 rr = fadd2(t, M);
@@ -201,6 +216,8 @@ __device__ __forceinline__ void p8_chunk(const uint32_t (&r)[32], float ck, floa
       float2 p = ffma2(C3, f, C2);
       p = ffma2(p, f, C1);
       p = ffma2(p, f, ONE);
+      // bits(rr) = 0x4B400000 + n with n = rint(t); shifting by 23 keeps n's low 9 bits,
+      // which is n << 23 modulo 2^32
       p.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(rr.x) << 23));
       p.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(rr.y) << 23));
       pp[h] = p;
@@ -237,6 +254,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
   auto bar_p = [&](int t) { return bar0 + 8u * (15 + t); };
   auto bar_pv = [&](int t) { return bar0 + 8u * (17 + t); };
   const uint32_t bar_done = bar0 + 8u * 19;
+  auto bar_sf = [&](int t) { return bar0 + 8u * (20 + t); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -293,6 +311,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       mbar_init(bar_s(t), 1);
       mbar_init(bar_p(t), 4);  // one arrival per softmax warp
       mbar_init(bar_pv(t), 1);
+      mbar_init(bar_sf(t), 4);  // one arrival per softmax warp: S region re-armed
     }
     mbar_init(bar_done, 1);
     fence_barrier_init();
@@ -364,7 +383,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const uint32_t d_tmem = tmem + kColS0 + 128u * t;
 #pragma unroll
         for (int s = 0; s < D / 32; ++s)
-          mma_i8_ss(d_tmem, aq + 2u * s, bk + 2u * s, kIdescS, s > 0 ? 1u : 0u);
+          mma_i8_ss(d_tmem, aq + 2u * s, bk + 2u * s, kIdescS, 1u);
         tc_commit(bar_s(t));
       };
       auto issue_pv = [&](int t, int vs) {
@@ -376,13 +395,17 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
           mma_f8_ts(d_tmem, a_tmem + 8u * s, bv + 2u * s, kIdescPV, s > 0 ? 1u : 0u);
         tc_commit(bar_pv(t));
       };
+      // S_t(j) accumulates onto the magic bit pattern the softmax warps wrote into the
+      // S region (re-armed after PV_t(j-1) consumed P_t(j-1)): wait for that first
       bool ok = mbar_wait(bar_q(), 0, 0x201) && mbar_wait(bar_kf(0), 0, 0x202);
-      if (ok) {
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (nkv[t] == 0) continue;
+        ok = mbar_wait(bar_sf(t), 0, 0x207 + t);
+        if (!ok) break;
         tc_fence_after();
-        for (int t = 0; t < 2; ++t)
-          if (nkv[t] > 0) issue_s(t, 0);
-        tc_commit(bar_ke(0));
+        issue_s(t, 0);
       }
+      if (ok) tc_commit(bar_ke(0));
       for (int j = 0; j < n_iter && ok; ++j) {
         const int vs = j % kVStages;
         bool v_ready = false, k_ready = false;
@@ -397,6 +420,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
           issue_pv(t, vs);
           if (jn < nkv[t]) {
             if (!k_ready) { ok = mbar_wait(bar_kf(ksn), (jn / kKStages) & 1, 0x206); k_ready = true; }
+            if (ok) ok = mbar_wait(bar_sf(t), jn & 1, 0x207 + t);
             if (!ok) break;
             tc_fence_after();
             issue_s(t, ksn);
@@ -434,25 +458,27 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                                   : 0.0f;
     const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kBlkK) + off / kBlkK;
 
+    // arm the S region: the first QK^T accumulates onto the magic bit pattern
+    if (ok && nkv[t] > 0) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_fill_magic32(tS + 32u * c);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_sf(t));
+    }
+
     for (int j = 0; j < nkv[t] && ok; ++j) {
       const float ck0 = __fmul_rn(__fmul_rn(sq, ksc[2 * j]), a.scale_log2);
       const float ck1 = __fmul_rn(__fmul_rn(sq, ksc[2 * j + 1]), a.scale_log2);
       const bool masked = (a.causal && j == qt[t]) || (j + 1) * kKvTile > n;
       const int kv0 = j * kKvTile;
+      auto dropped = [&](int key) { return key >= n || (a.causal && key > grow); };
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s(t), j & 1, 0x301 + t));
       if (!ok) break;
       tc_fence_after();
 
-      // masked keys (past the sequence end or above the causal diagonal) read as NaN
-      auto mask_chunk = [&](uint32_t (&r)[32], int c) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int key = kv0 + 32 * c + i;
-          if (key >= n || (a.causal && key > grow)) r[i] = 0xFFFFFFFFu;
-        }
-      };
-
-      // pass 1: largest score of each 64-key half
+      // pass 1: largest score of each 64-key half (masked keys read as 0 < every valid value)
       float hmax[2];
       {
         uint32_t ra[32], rb[32];
@@ -461,78 +487,39 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
           tmem_ld32(tS + 64u * h, ra);
           tmem_ld32(tS + 64u * h + 32u, rb);
           tmem_wait_ld_tied(ra, rb);
-          if (masked) { mask_chunk(ra, 2 * h); mask_chunk(rb, 2 * h + 1); }
-          hmax[h] = max_nonneg32(rb, max_nonneg32(ra, __uint_as_float(0xFFFFFFFFu)));
-        }
-      }
-      int imax[2];
+          if (masked) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        imax[h] = static_cast<int>(__float_as_uint(hmax[h]));
-        // a row with no non-negative score in this half needs the exact integer max; the
-        // TMEM reload is warp-collective, so the whole warp takes this branch together
-        if (__any_sync(0xffffffffu, isnan(hmax[h]))) {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(tS + 64u * h, ra);
-          tmem_ld32(tS + 64u * h + 32u, rb);
-          tmem_wait_ld_tied(ra, rb);
-          int mx = INT_MIN;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int k0 = kv0 + 64 * h + i, k1 = k0 + 32;
-            const bool d0 = masked && (k0 >= n || (a.causal && k0 > grow));
-            const bool d1 = masked && (k1 >= n || (a.causal && k1 > grow));
-            mx = d0 ? mx : max(mx, static_cast<int>(ra[i]));
-            mx = d1 ? mx : max(mx, static_cast<int>(rb[i]));
+            for (int i = 0; i < 32; ++i) {
+              if (dropped(kv0 + 64 * h + i)) ra[i] = 0u;
+              if (dropped(kv0 + 64 * h + 32 + i)) rb[i] = 0u;
+            }
           }
-          if (isnan(hmax[h])) imax[h] = mx;
+          hmax[h] = max32(rb, max32(ra, 0.0f));
         }
       }
-      const float mt = fmaxf(imax[0] == INT_MIN ? -INFINITY : __fmul_rn(static_cast<float>(imax[0]), ck0),
-                             imax[1] == INT_MIN ? -INFINITY : __fmul_rn(static_cast<float>(imax[1]), ck1));
+      // an all-masked half leaves 0; valid values are at least 12582912 - 2^21
+      const float mt = fmaxf(hmax[0] > 1.0e6f ? __fmul_rn(__fsub_rn(hmax[0], kMagic), ck0) : -INFINITY,
+                             hmax[1] > 1.0e6f ? __fmul_rn(__fsub_rn(hmax[1], kMagic), ck1) : -INFINITY);
       const float m_new = fmaxf(m, mt);
       const float alpha = ex2(m - m_new);
       const float nbias = __fsub_rn(kLog2_448, m_new);
-      const float cb0 = __fsub_rn(nbias, __fmul_rn(12582912.0f, ck0));
-      const float cb1 = __fsub_rn(nbias, __fmul_rn(12582912.0f, ck1));
 
-      // pass 2: p = 448 * 2^(u - m'), running sum, e4m3 P8 into TMEM over the S columns
+      // pass 2: p = 448 * 2^(u - m'), running sum, e4m3 P8 into TMEM columns 0-31,
+      // columns 32-127 re-armed with the magic pattern once read
       float2 acc = make_float2(0.0f, 0.0f);
       {
         uint32_t ra[32], rb[32], w[8];
         auto finish = [&](uint32_t (&r)[32], int c) {
           if (masked) {
-            float2 dummy = make_float2(0.0f, 0.0f);
-            p8_chunk(r, c < 2 ? ck0 : ck1, c < 2 ? cb0 : cb1, dummy, w);
-            // recompute with masked entries zeroed (tiles on the diagonal / sequence tail)
-            float2 acc_m = make_float2(0.0f, 0.0f);
+            // a masked key reads as -inf: t becomes the -125 clamp, p = 2^-125, whose
+            // e4m3 code is 0 and which vanishes in l (l >= ~448, its fp32 unit is 2^-15)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              uint32_t code = w[i];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int key = kv0 + 32 * c + 4 * i + e;
-                if (key >= n || (a.causal && key > grow)) code &= ~(0xFFu << (8 * e));
-              }
-              w[i] = code;
-            }
-            // the running sum needs the unquantized values of the kept keys only
-            {
-              const float ck = c < 2 ? ck0 : ck1, cb = c < 2 ? cb0 : cb1;
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int key = kv0 + 32 * c + i;
-                const float tt = __fmaf_rn(__int_as_float(static_cast<int>(r[i]) + 0x4B400000), ck, cb);
-                const float pv = exp2_poly(tt);
-                if (!(key >= n || (a.causal && key > grow))) acc_m.x = __fadd_rn(acc_m.x, pv);
-              }
-            }
-            acc = fadd2(acc, acc_m);
-            (void)dummy;
-          } else {
-            p8_chunk(r, c < 2 ? ck0 : ck1, c < 2 ? cb0 : cb1, acc, w);
+            for (int i = 0; i < 32; ++i)
+              if (dropped(kv0 + 32 * c + i)) r[i] = 0xFF800000u;
           }
+          p8_chunk(r, c < 2 ? ck0 : ck1, nbias, acc, w);
           tmem_st8(tS + 8u * c, w);
+          if (c > 0) tmem_fill_magic32(tS + 32u * c);
         };
         tmem_ld32(tS, ra);
         tmem_wait_ld_tied(ra);
@@ -558,6 +545,13 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       ok = __all_sync(0xffffffffu, mbar_wait(bar_pv(t), j & 1, 0x303 + t));
       if (!ok) break;
       tc_fence_after();
+      if (j + 1 < nkv[t]) {  // P consumed: re-arm columns 0-31 for the next QK^T
+        tmem_fill_magic32(tS);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_sf(t));
+      }
       {
         const float2 al = make_float2(alpha, alpha);
         uint32_t ra[32], rb[32];
