@@ -382,12 +382,13 @@ def fma_f32(a, b, c) -> np.ndarray:
 
 
 def exp2_f32(t) -> np.ndarray:
-    """2^t in fp32 operations: t clamped at -125, n = rint(t) by magic-number
-    rounding, f = t - n in [-1/2, 1/2], Horner polynomial 1 + c1 f + c2 f^2 + c3 f^3
-    (fp32 FMAs), and n added to the exponent field."""
-    t = np.maximum(np.asarray(t, dtype=np.float32), np.float32(-125.0))
+    """2^t in fp32 operations: r = t + 1.5*2^23 rounds t to n = rint(t) (magic-number
+    rounding), f = t - (r - 1.5*2^23) in [-1/2, 1/2], Horner polynomial
+    1 + c1 f + c2 f^2 + c3 f^3 (fp32 FMAs), and n, clamped below at -125 so the
+    result stays a normal number, added to the exponent field."""
+    t = np.asarray(t, dtype=np.float32)
     r = (t + MAGIC_F32).astype(np.float32)
-    n = r.view(np.int32) - np.int32(0x4B400000)
+    n = np.maximum(r.view(np.int32), np.int32(0x4B400000 - 125)) - np.int32(0x4B400000)
     f = (t - (r - MAGIC_F32).astype(np.float32)).astype(np.float32)
     c0, c1, c2, c3 = EXP2_COEF_F32
     p = fma_f32(c3, f, c2)

@@ -6,7 +6,9 @@ import ctypes
 import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libsage.so")
+# SAGE_LIB_PATH may name another build of the same library (e.g. one built with
+# different compile options); the default is the in-tree build.
+LIB_PATH = os.environ.get("SAGE_LIB_PATH") or os.path.join(_PKG, "libsage.so")
 
 SAGE_OK = 0
 SAGE_ERR_INVALID_ARGUMENT = 1

@@ -93,38 +93,39 @@ __device__ __forceinline__ float ex2(float x) {
 
 // 2^t in plain IEEE fp32 operations, so that the P8 code it decides can be
 // reproduced exactly on any host: Cody-Waite split t = n + f with n = rint(t)
-// (magic-number rounding) and f in [-1/2, 1/2], a degree-3 polynomial for 2^f
-// (coefficients fitted for minimal relative error with the constant term fixed
-// at 1; max relative error 1.0e-4), and n added to the exponent field.  t is
-// clamped at -125 so the result stays a normal number.
+// taken by magic-number rounding (r = t + 1.5 * 2^23, bits(r) = 0x4B400000 + n)
+// and f = t - (r - 1.5 * 2^23) in [-1/2, 1/2], a degree-3 polynomial for 2^f
+// (coefficients fitted for minimal relative error with the constant term fixed at
+// 1; max relative error 1.0e-4), and n added to the exponent field, clamped below
+// at -125 so the result stays a normal number.
 constexpr float kExp2C1 = 0.693282962f;   // 0x3f317afe
 constexpr float kExp2C2 = 0.242211089f;   // 0x3e78062f
 constexpr float kExp2C3 = 0.0550086424f;  // 0x3d6150be
+constexpr int kExpClampBits = 0x4B400000 - 125;
 __device__ __forceinline__ float exp2_poly(float t) {
-  t = fmaxf(t, -125.0f);
   const float r = __fadd_rn(t, 12582912.0f);
-  const int n = __float_as_int(r) - 0x4B400000;
   const float f = __fsub_rn(t, __fsub_rn(r, 12582912.0f));
   float p = __fmaf_rn(kExp2C3, f, kExp2C2);
   p = __fmaf_rn(p, f, kExp2C1);
   p = __fmaf_rn(p, f, 1.0f);
-  return __int_as_float(__float_as_int(p) + (n << 23));
+  const int rb = max(__float_as_int(r), kExpClampBits);
+  return __int_as_float(__float_as_int(p) + rb * (1 << 23));
 }
 
-// ---- packed fp32 pair arithmetic (one instruction per two values)
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  float2 d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;"
-      : "=l"(reinterpret_cast<uint64_t&>(d))
-      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)),
-        "l"(reinterpret_cast<const uint64_t&>(c)));
+// ---- packed fp32 pair arithmetic (one instruction per two values); element 0 of a
+// pair is .x, handed to the f32x2 instructions as the low half of a 64-bit register.
+using f2 = float2;
+__device__ __forceinline__ f2 f2_make(float lo, float hi) { return make_float2(lo, hi); }
+__device__ __forceinline__ float f2_lo(f2 a) { return a.x; }
+__device__ __forceinline__ float f2_hi(f2 a) { return a.y; }
+__device__ __forceinline__ f2 f2_fma(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(reinterpret_cast<uint64_t&>(d)) : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)), "l"(reinterpret_cast<const uint64_t&>(c)));
   return d;
 }
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-  float2 d;
-  asm("add.rn.f32x2 %0, %1, %2;"
-      : "=l"(reinterpret_cast<uint64_t&>(d))
-      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)));
+__device__ __forceinline__ f2 f2_add(f2 a, f2 b) {
+  f2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(reinterpret_cast<uint64_t&>(d)) : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)));
   return d;
 }
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -158,7 +159,9 @@ __device__ __forceinline__ void tmem_wait_ld_tied(uint32_t (&a)[32], uint32_t (&
                :
                : "memory");
 }
-
+__device__ __forceinline__ f2 pair_of(const uint32_t (&r)[32], int k) {
+  return f2_make(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+}
 // The S region is pre-filled with kMagicBits (the fp32 1.5 * 2^23 = 12582912) and the
 // INT8 MMAs accumulate onto it, so TMEM returns bits(12582912 + S): an fp32 whose
 // value is exactly 12582912 + S for |S| < 2^22 (|S| <= d * 127^2 here).  Those values
@@ -193,37 +196,40 @@ __device__ __forceinline__ float max32(const uint32_t (&r)[32], float acc) {
 // P for 32 keys of one 64-key half: S = (12582912 + S) - 12582912 (exact),
 // t = fma(S, ck, log2 448 - m'), p = exp2_poly(t) evaluated two values per
 // instruction (the same fp32 operations as exp2_poly).  Returns the e4m3 codes
-// packed four per word and adds p into acc.
-__device__ __forceinline__ void p8_chunk(const uint32_t (&r)[32], float ck, float nb, float2& acc,
-                                         uint32_t (&w)[8]) {
-  const float2 CK = make_float2(ck, ck), NB = make_float2(nb, nb);
-  const float2 M = make_float2(kMagic, kMagic), NM = make_float2(-kMagic, -kMagic);
-  const float2 NEG1 = make_float2(-1.0f, -1.0f), ONE = make_float2(1.0f, 1.0f);
-  const float2 C1 = make_float2(kExp2C1, kExp2C1), C2 = make_float2(kExp2C2, kExp2C2);
-  const float2 C3 = make_float2(kExp2C3, kExp2C3);
+// packed four per word and adds p into acc.  With kMasked, key i is kept only
+// when bit i of `keep` is set; dropped keys get p = 0.
+template <bool kMasked>
+__device__ __forceinline__ void p8_chunk(const uint32_t (&r)[32], float ck, float nb, f2& acc,
+                                         uint32_t (&w)[8], uint32_t keep) {
+  const f2 CK = f2_make(ck, ck), NB = f2_make(nb, nb);
+  const f2 M = f2_make(kMagic, kMagic), NM = f2_make(-kMagic, -kMagic);
+  const f2 NEG1 = f2_make(-1.0f, -1.0f), ONE = f2_make(1.0f, 1.0f);
+  const f2 C1 = f2_make(kExp2C1, kExp2C1), C2 = f2_make(kExp2C2, kExp2C2);
+  const f2 C3 = f2_make(kExp2C3, kExp2C3);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    float2 pp[2];
+    f2 pp[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int e = 4 * i + 2 * h;
-      const float2 x = fadd2(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), NM);
-      float2 t = ffma2(x, CK, NB);
-      t.x = fmaxf(t.x, -125.0f);
-      t.y = fmaxf(t.y, -125.0f);
-      const float2 rr = fadd2(t, M);
-      const float2 f = ffma2(fadd2(rr, NM), NEG1, t);
-      float2 p = ffma2(C3, f, C2);
-      p = ffma2(p, f, C1);
-      p = ffma2(p, f, ONE);
-      // bits(rr) = 0x4B400000 + n with n = rint(t); shifting by 23 keeps n's low 9 bits,
-      // which is n << 23 modulo 2^32
-      p.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(rr.x) << 23));
-      p.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(rr.y) << 23));
-      pp[h] = p;
+      const f2 t = f2_fma(f2_add(pair_of(r, 2 * i + h), NM), CK, NB);
+      const f2 rr = f2_add(t, M);
+      const f2 f = f2_fma(f2_add(rr, NM), NEG1, t);
+      f2 p = f2_fma(C3, f, C2);
+      p = f2_fma(p, f, C1);
+      p = f2_fma(p, f, ONE);
+      // bits(rr) = 0x4B400000 + n: max() clamps n at -125, and bits << 23 is n << 23
+      // modulo 2^32
+      uint32_t lo = __float_as_uint(p.x) + (static_cast<uint32_t>(max(__float_as_int(rr.x), kExpClampBits)) << 23);
+      uint32_t hi = __float_as_uint(p.y) + (static_cast<uint32_t>(max(__float_as_int(rr.y), kExpClampBits)) << 23);
+      if (kMasked) {
+        const int e = 4 * i + 2 * h;
+        lo = ((keep >> e) & 1u) ? lo : 0u;
+        hi = ((keep >> (e + 1)) & 1u) ? hi : 0u;
+      }
+      pp[h] = f2_make(__uint_as_float(lo), __uint_as_float(hi));
     }
-    acc = fadd2(acc, fadd2(pp[0], pp[1]));
-    w[i] = e4m3x2(pp[0].x, pp[0].y) | (e4m3x2(pp[1].x, pp[1].y) << 16);
+    acc = f2_add(acc, f2_add(pp[0], pp[1]));
+    w[i] = e4m3x2(f2_lo(pp[0]), f2_hi(pp[0])) | (e4m3x2(f2_lo(pp[1]), f2_hi(pp[1])) << 16);
   }
 }
 
@@ -361,12 +367,12 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       }
       // drain: the most recent load of every stage has landed before the CTA can exit
       const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(bar_q(), 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
+      while (!mbar_try_wait_sleep(bar_q(), 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
       for (int jj = max(0, nk - kKStages); jj < nk; ++jj)
-        while (!mbar_try_wait(bar_kf(jj % kKStages), (jj / kKStages) & 1) &&
+        while (!mbar_try_wait_sleep(bar_kf(jj % kKStages), (jj / kKStages) & 1) &&
                global_timer_ns() - t0 < kWaitLimitNs) {}
       for (int jj = max(0, nv - kVStages); jj < nv; ++jj)
-        while (!mbar_try_wait(bar_vf(jj % kVStages), (jj / kVStages) & 1) &&
+        while (!mbar_try_wait_sleep(bar_vf(jj % kVStages), (jj / kVStages) & 1) &&
                global_timer_ns() - t0 < kWaitLimitNs) {}
     }
   } else if (warp == 1) {
@@ -434,7 +440,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       // every MMA issued by this thread has completed before TMEM is released
       tc_commit(bar_done);
       const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(bar_done, 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
+      while (!mbar_try_wait_sleep(bar_done, 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
     }
    }
   } else {
@@ -448,7 +454,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const uint32_t tS = tmem + lane_base + kColS0 + 128u * t;
     const uint32_t tPV = tmem + lane_base + kColPV0 + 128u * t;
 
-    float2 o2[D / 2];
+    f2 o2[D / 2];  // running output, columns (2c, 2c+1) in pair c
 #pragma unroll
     for (int c = 0; c < D / 2; ++c) o2[c] = make_float2(0.0f, 0.0f);
     float m = -INFINITY, l = 0.0f;
@@ -506,18 +512,20 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
       // pass 2: p = 448 * 2^(u - m'), running sum, e4m3 P8 into TMEM columns 0-31,
       // columns 32-127 re-armed with the magic pattern once read
-      float2 acc = make_float2(0.0f, 0.0f);
+      f2 acc = make_float2(0.0f, 0.0f);
       {
-        uint32_t ra[32], rb[32], w[8];
+        uint32_t ra[32], rb[32];
+        uint32_t w[8];
         auto finish = [&](uint32_t (&r)[32], int c) {
+          const float ck = c < 2 ? ck0 : ck1;
           if (masked) {
-            // a masked key reads as -inf: t becomes the -125 clamp, p = 2^-125, whose
-            // e4m3 code is 0 and which vanishes in l (l >= ~448, its fp32 unit is 2^-15)
+            uint32_t keep = 0u;
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (dropped(kv0 + 32 * c + i)) r[i] = 0xFF800000u;
+            for (int i = 0; i < 32; ++i) keep |= dropped(kv0 + 32 * c + i) ? 0u : (1u << i);
+            p8_chunk<true>(r, ck, nbias, acc, w, keep);
+          } else {
+            p8_chunk<false>(r, ck, nbias, acc, w, 0u);
           }
-          p8_chunk(r, c < 2 ? ck0 : ck1, nbias, acc, w);
           tmem_st8(tS + 8u * c, w);
           if (c > 0) tmem_fill_magic32(tS + 32u * c);
         };
@@ -538,7 +546,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_p(t));
-      l = l * alpha + (acc.x + acc.y);
+      l = l * alpha + (f2_lo(acc) + f2_hi(acc));
       m = m_new;
 
       // two-level accumulation: O = alpha * O + PV_blk (PV_blk fresh in TMEM for this tile)
@@ -553,13 +561,11 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         if (lane == 0) mbar_arrive(bar_sf(t));
       }
       {
-        const float2 al = make_float2(alpha, alpha);
+        const f2 al = f2_make(alpha, alpha);
         uint32_t ra[32], rb[32];
         auto accum = [&](const uint32_t (&r)[32], int c) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            o2[16 * c + i] = ffma2(o2[16 * c + i], al,
-                                   make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])));
+          for (int i = 0; i < 16; ++i) o2[16 * c + i] = f2_fma(o2[16 * c + i], al, pair_of(r, i));
         };
         tmem_ld32(tPV, ra);
         tmem_wait_ld_tied(ra);
@@ -584,8 +590,8 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         float* dst = reinterpret_cast<float*>(a.out) + orow;
 #pragma unroll
         for (int c = 0; c < D; c += 4) {
-          float4 v = make_float4(o2[c / 2].x * vs[c] * inv_l, o2[c / 2].y * vs[c + 1] * inv_l,
-                                 o2[c / 2 + 1].x * vs[c + 2] * inv_l, o2[c / 2 + 1].y * vs[c + 3] * inv_l);
+          float4 v = make_float4(f2_lo(o2[c / 2]) * vs[c] * inv_l, f2_hi(o2[c / 2]) * vs[c + 1] * inv_l,
+                                 f2_lo(o2[c / 2 + 1]) * vs[c + 2] * inv_l, f2_hi(o2[c / 2 + 1]) * vs[c + 3] * inv_l);
           *reinterpret_cast<float4*>(dst + c) = v;
         }
       } else if (a.out_dtype == 1) {
@@ -594,7 +600,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         for (int c = 0; c < D; c += 8) {
           __align__(16) __nv_bfloat16 h8[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) h8[i] = __float2bfloat16_rn(((i & 1) ? o2[(c + i) / 2].y : o2[(c + i) / 2].x) * vs[c + i] * inv_l);
+          for (int i = 0; i < 8; ++i) h8[i] = __float2bfloat16_rn(((i & 1) ? f2_hi(o2[(c + i) / 2]) : f2_lo(o2[(c + i) / 2])) * vs[c + i] * inv_l);
           *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<const uint4*>(h8);
         }
       } else {
@@ -603,7 +609,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         for (int c = 0; c < D; c += 8) {
           __align__(16) __half h8[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) h8[i] = __float2half_rn(((i & 1) ? o2[(c + i) / 2].y : o2[(c + i) / 2].x) * vs[c + i] * inv_l);
+          for (int i = 0; i < 8; ++i) h8[i] = __float2half_rn(((i & 1) ? f2_hi(o2[(c + i) / 2]) : f2_lo(o2[(c + i) / 2])) * vs[c + i] * inv_l);
           *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<const uint4*>(h8);
         }
       }

@@ -80,15 +80,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0u;
 }
 
+// try_wait that may suspend the thread until the phase completes (or about
+// kSuspendHintNs elapses): used where a thread only drains before exiting.  The
+// hot-path waits below use the plain form, whose wake-up latency measured lower.
+constexpr uint32_t kSuspendHintNs = 0x989680u;  // 10 ms
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0u;
+}
+
 // Wait for phase `parity` of an mbarrier, at most kWaitLimitNs.  On timeout the
 // watchdog word records `site` and false is returned; the caller must stop.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (watchdog_tripped()) return false;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       watchdog_trip(site);

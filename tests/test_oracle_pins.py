@@ -410,6 +410,9 @@ def test_exp2_f32_accuracy_and_exact_powers():
     assert np.array_equal(orc.exp2_f32(ti), np.exp2(ti))
     assert np.all(np.diff(orc.exp2_f32(np.linspace(-3, 3, 10001).astype(np.float32))) >= 0)
     assert orc.exp2_f32(np.float32([-1000.0]))[0] == np.float32(2.0 ** -125)
+    # below -125 the exponent step is clamped: tiny, normal, never zero or garbage
+    tiny = orc.exp2_f32(np.float32([-125.6, -300.3, -4.0e6, -3.0e9]))
+    assert np.all((tiny > 2.0 ** -127) & (tiny < 2.0 ** -123))
 
 
 @pytest.mark.parametrize("causal", [False, True])
