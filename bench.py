@@ -279,7 +279,25 @@ def run_sage(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out.numel() * out.element_size(),
                "ms_per_step": e_ms}
 
-    bf16, bf16_sus, _, src = peaks()
+    # ---- quantization kernels alone: algorithmic HBM bytes / time
+    def timed(fn, reps=5):
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+    qk_ms = timed(lambda: api.quant_qk(q, k, "HND", problem=p, out=z, workspace=ws_qk))
+    v_ms = timed(lambda: api.quant_v(v, z, workspace=ws_v))
+    elems_q = q.numel()
+    elems_kv = k.numel()
+    qk_bytes = 3.0 * elems_q + 5.0 * elems_kv   # Q: read 2 + write 1; K: 2 reads of 2 + write 1
+    v_bytes = 5.0 * elems_kv                      # V: 2 reads of 2 + write 1
+
+    bf16, bf16_sus, hbm, src = peaks()
     peak = bf16 * NOMINAL_INT8_OVER_BF16
     achieved = ops / (attn_mean * 1e-3) / 1e12
     traffic = None
@@ -307,6 +325,12 @@ def run_sage(args):
                                                if bf16_sus else None),
                          "frac_of_datasheet_4500": achieved / 4500.0},
             "e2e": e2e,
+            "quant": {"unit": "GB/s", "hbm_peak": hbm,
+                      "quant_qk": {"ms": qk_ms, "achieved": qk_bytes / (qk_ms * 1e-3) / 1e9,
+                                   "frac": qk_bytes / (qk_ms * 1e-3) / 1e9 / hbm,
+                                   "bytes": qk_bytes},
+                      "quant_v": {"ms": v_ms, "achieved": v_bytes / (v_ms * 1e-3) / 1e9,
+                                  "frac": v_bytes / (v_ms * 1e-3) / 1e9 / hbm, "bytes": v_bytes}},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
         }
