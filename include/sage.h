@@ -18,7 +18,8 @@
  * ---------------------------------
  * - Pointers are device memory owned by the caller unless marked "host".  The
  *   library allocates no device memory and keeps no state between calls except
- *   the device watchdog word read by sage_poll_device_status().
+ *   the device watchdog word read by sage_poll_device_status() and the scratch
+ *   array of sage_quant_qk_noalloc.
  * - Work is enqueued on `stream` (a cudaStream_t); calls return once enqueued.
  * - Errors: argument problems return SAGE_ERR_INVALID_ARGUMENT or
  *   SAGE_ERR_UNSUPPORTED before anything is enqueued; a failed launch returns
@@ -64,7 +65,8 @@ typedef enum {
   SAGE_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size, misaligned, too small workspace */
   SAGE_ERR_UNSUPPORTED = 2,      /* head_dim not 64/128, unknown dtype, device not sm_100 */
   SAGE_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed */
-  SAGE_ERR_DEVICE_TIMEOUT = 4    /* a kernel's bounded wait ran out (see sage_poll_device_status) */
+  SAGE_ERR_DEVICE_TIMEOUT = 4,   /* a kernel's bounded wait ran out (see sage_poll_device_status) */
+  SAGE_ERR_TOO_LARGE = 5         /* the problem needs more scratch than sage_quant_qk_noalloc holds */
 } sage_status_t;
 
 typedef enum { SAGE_FP16 = 0, SAGE_BF16 = 1, SAGE_FP32 = 2 } sage_dtype_t;
@@ -111,6 +113,30 @@ sage_status_t sage_quant_qk(const sage_problem_t* p,
                             int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
                             float* k_mean, void* workspace, size_t workspace_bytes,
                             sage_stream_t stream);
+
+/*
+ * sage_quant_qk_noalloc - sage_quant_qk without a caller workspace.
+ * The pages describe no counterpart: this is a deployment convenience.  It is for
+ * callers that cannot allocate device memory when they quantize (a framework hook
+ * whose allocator is locked, a plugin that may only use the tensors it is given, a
+ * pipeline whose buffers are all reserved up front).  Arguments, outputs and
+ * results are those of sage_quant_qk; the fp64 column-sum scratch lives instead in
+ * a library-owned device array of SAGE_NOALLOC_SCRATCH_BYTES (8 MiB) on every GPU
+ * that loads the library, kept until the process exits.
+ * - Returns SAGE_ERR_TOO_LARGE, before enqueuing anything, when the problem needs
+ *   more scratch than that (sizes.workspace_qk > SAGE_NOALLOC_SCRATCH_BYTES).
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call before
+ *   any stream capture.  It allocates nothing (no cudaMalloc / cudaFree).
+ * - All calls share the array, which keeps the last call's contents (nothing in it
+ *   needs clearing); calls that overlap on the GPU, from any stream or thread, race.
+ */
+#define SAGE_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+sage_status_t sage_quant_qk_noalloc(const sage_problem_t* p,
+                                    const void* q, const int64_t q_strides[3],
+                                    const void* k, const int64_t k_strides[3],
+                                    int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
+                                    float* k_mean, sage_stream_t stream);
 
 /*
  * sage_quant_v - per-channel FP8 e4m3 quantization of V, written transposed.

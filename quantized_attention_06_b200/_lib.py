@@ -15,12 +15,15 @@ SAGE_ERR_INVALID_ARGUMENT = 1
 SAGE_ERR_UNSUPPORTED = 2
 SAGE_ERR_CUDA = 3
 SAGE_ERR_DEVICE_TIMEOUT = 4
+SAGE_ERR_TOO_LARGE = 5
+NOALLOC_SCRATCH_BYTES = 8 << 20  # SAGE_NOALLOC_SCRATCH_BYTES
 
 SAGE_FP16, SAGE_BF16, SAGE_FP32 = 0, 1, 2
 
 EXPORTS = (
     "sage_buffer_sizes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd",
-    "sage_debug_qk_int32", "sage_poll_device_status", "sage_status_string",
+    "sage_debug_qk_int32", "sage_poll_device_status", "sage_quant_qk_noalloc",
+    "sage_status_string",
 )
 
 
@@ -66,6 +69,7 @@ def lib() -> ctypes.CDLL:
     L.sage_buffer_sizes.argtypes = [P(SageProblem), P(SageSizes)]
     L.sage_quant_qk.argtypes = [P(SageProblem), vp, i64p, vp, i64p, vp, vp, vp, vp, vp, vp, sz, vp]
     L.sage_quant_v.argtypes = [P(SageProblem), vp, i64p, vp, vp, vp, sz, vp]
+    L.sage_quant_qk_noalloc.argtypes = [P(SageProblem), vp, i64p, vp, i64p, vp, vp, vp, vp, vp, vp]
     L.sage_attn_fwd.argtypes = [P(SageProblem), vp, vp, vp, vp, vp, vp, ctypes.c_float,
                                 ctypes.c_int, vp, ctypes.c_int, i64p, vp, vp]
     L.sage_debug_qk_int32.argtypes = [P(SageProblem), vp, vp, ctypes.c_int, ctypes.c_int, vp, vp]

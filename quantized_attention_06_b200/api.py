@@ -22,8 +22,8 @@ import torch
 
 from . import _lib as L
 
-__all__ = ["Problem", "Quantized", "quant_qk", "quant_v", "attn_fwd", "sageattn",
-           "debug_qk_int32", "poll_device_status"]
+__all__ = ["Problem", "Quantized", "quant_qk", "quant_qk_noalloc", "quant_v", "attn_fwd",
+           "sageattn", "debug_qk_int32", "poll_device_status"]
 
 _IN_DTYPES = {torch.float16: L.SAGE_FP16, torch.bfloat16: L.SAGE_BF16}
 _OUT_DTYPES = {torch.float16: L.SAGE_FP16, torch.bfloat16: L.SAGE_BF16, torch.float32: L.SAGE_FP32}
@@ -139,6 +139,31 @@ def quant_qk(q, k, tensor_layout="HND", cu_seqlens=None, problem=None, out: Quan
         _ptr(z.q8), _ptr(z.q_scale), _ptr(z.k8), _ptr(z.k_scale), _ptr(z.k_mean),
         _ptr(ws), ws.numel() * ws.element_size(), _stream())
     L.check("sage_quant_qk", st)
+    return z
+
+
+def quant_qk_noalloc(q, k, tensor_layout="HND", cu_seqlens=None, problem=None,
+                     out: Quantized = None) -> Quantized:
+    """quant_qk without a workspace (sage_quant_qk_noalloc), for callers that cannot
+    allocate device memory when they quantize.  The scratch comes from a fixed
+    library-owned device array; ``out`` should then hold preallocated outputs.
+    Calls that overlap on the GPU race on that shared scratch."""
+    _require_cuda(q, k)
+    p = problem or Problem.from_tensors(q, k, tensor_layout, cu_seqlens)
+    z = out or Quantized(p, tensor_layout)
+    dev = q.device
+    d, tp = p.head_dim, p.t_pad
+    if z.q8 is None:
+        z.q8 = torch.empty((p.heads_q, tp, d), dtype=torch.int8, device=dev)
+        z.q_scale = torch.empty((p.heads_q, tp // 128), dtype=torch.float32, device=dev)
+        z.k8 = torch.empty((p.heads_kv, tp, d), dtype=torch.int8, device=dev)
+        z.k_scale = torch.empty((p.heads_kv, tp // 64), dtype=torch.float32, device=dev)
+        z.k_mean = torch.empty((p.batch, p.heads_kv, d), dtype=torch.float32, device=dev)
+    st = L.lib().sage_quant_qk_noalloc(
+        ctypes.byref(p.c), _ptr(q), _strides(q, tensor_layout, p.varlen),
+        _ptr(k), _strides(k, tensor_layout, p.varlen),
+        _ptr(z.q8), _ptr(z.q_scale), _ptr(z.k8), _ptr(z.k_scale), _ptr(z.k_mean), _stream())
+    L.check("sage_quant_qk_noalloc", st)
     return z
 
 

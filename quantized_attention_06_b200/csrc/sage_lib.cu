@@ -210,6 +210,7 @@ const char* sage_status_string(sage_status_t s) {
     case SAGE_ERR_UNSUPPORTED: return "SAGE_ERR_UNSUPPORTED";
     case SAGE_ERR_CUDA: return "SAGE_ERR_CUDA";
     case SAGE_ERR_DEVICE_TIMEOUT: return "SAGE_ERR_DEVICE_TIMEOUT";
+    case SAGE_ERR_TOO_LARGE: return "SAGE_ERR_TOO_LARGE";
   }
   return "SAGE_ERR_UNKNOWN";
 }
@@ -386,3 +387,77 @@ sage_status_t sage_poll_device_status(sage_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ====================================================================== scratch-free sage_quant_qk
+// sage_quant_qk writes per-block fp64 column sums of K into a workspace the caller
+// allocates.  Some callers cannot allocate device memory at the moment they
+// quantize: code running inside a framework hook whose caching allocator is
+// locked or mid-teardown, plugins that may only touch the tensors they are handed,
+// and pipelines whose every device buffer is reserved up front.  For them
+// sage_quant_qk_noalloc takes that scratch from the array below instead.
+//
+// The array is a fixed, modest size held by every GPU that loads this library
+// until the process exits; problems that need more are rejected.  Host code may
+// not use the array's name as a device address (it is a host-side stand-in), so
+// the device address is looked up with cudaGetSymbolAddress, once per device, on
+// that device's first call.  All calls share the array and it keeps the last
+// call's contents; every word a call reads was written earlier in the same call,
+// so nothing needs clearing, but calls that overlap on the GPU race on it.
+static __device__ __align__(256) unsigned char g_quant_qk_scratch[SAGE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_quant_qk_scratch on the current device (looked up once).
+sage_status_t static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SAGE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_quant_qk_scratch) != cudaSuccess || ptr == nullptr)
+      return SAGE_ERR_CUDA;
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return SAGE_OK;
+}
+
+}  // namespace
+
+extern "C" sage_status_t sage_quant_qk_noalloc(const sage_problem_t* p, const void* q,
+                                               const int64_t q_strides[3], const void* k,
+                                               const int64_t k_strides[3], int8_t* q8,
+                                               float* q_scale, int8_t* k8, float* k_scale,
+                                               float* k_mean, sage_stream_t stream) {
+  static thread_local SeqVarlen var;
+  Layout L;
+  sage_status_t st = plan(p, L, &var);
+  if (st != SAGE_OK) return st;
+  sage_sizes_t sz;
+  sage_buffer_sizes(p, &sz);
+  if (!q || !k || !q8 || !q_scale || !k8 || !k_scale || !k_mean) return SAGE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q8) || !aligned16(k8))
+    return SAGE_ERR_INVALID_ARGUMENT;
+  if (!strides_ok(p, q_strides, 2) || !strides_ok(p, k_strides, 2)) return SAGE_ERR_INVALID_ARGUMENT;
+  if (sz.workspace_qk > SAGE_NOALLOC_SCRATCH_BYTES) return SAGE_ERR_TOO_LARGE;
+  if ((st = device_ok()) != SAGE_OK) return st;
+  void* ws = nullptr;
+  if ((st = static_scratch(&ws)) != SAGE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+#define SAGE_QK(T, D)                                                                           \
+  return L.varlen ? launch_quant_qk<T, D>(*L.var, p, L.t_pad, q, q_strides, k, k_strides, q8,    \
+                                          q_scale, k8, k_scale, k_mean, ws, s)                   \
+                  : launch_quant_qk<T, D>(L.dense, p, L.t_pad, q, q_strides, k, k_strides, q8,   \
+                                          q_scale, k8, k_scale, k_mean, ws, s)
+  if (p->dtype == SAGE_FP16) {
+    if (p->head_dim == 128) { SAGE_QK(__half, 128); } else { SAGE_QK(__half, 64); }
+  } else {
+    if (p->head_dim == 128) { SAGE_QK(__nv_bfloat16, 128); } else { SAGE_QK(__nv_bfloat16, 64); }
+  }
+#undef SAGE_QK
+}
