@@ -7,24 +7,29 @@
 // variable lengths); glossary page "SageAttention(セージアテンション)" (FlashAttention-
 // compatible online softmax).
 //
-// CTA = one (sequence, query head, pair of 128-row Q tiles).  12 warps in three
-// warpgroups; the producer warpgroup gives registers to the softmax warpgroups
-// (setmaxnreg: 128 x 40 + 256 x 232 = 384 x 168, the launch allocation):
-//   warp 0      TMA producer: both Q tiles once, then K / V tiles into 3-stage rings
-//   warp 1      TMEM owner and MMA issuer (one thread):
-//                 S_t  = Q8_t K8^T      tcgen05.mma kind::i8     -> TMEM s32 [128 x 128]
-//                 PV_t = P8_t V8       tcgen05.mma kind::f8f6f4 (A = P8 in TMEM) -> TMEM f32 [128 x d]
-//   warps 2-3   idle
-//   warps 4-7   softmax + correction for Q tile 0 (one thread per query row)
-//   warps 8-11  softmax + correction for Q tile 1
-// TMEM columns: [0,128) S/P of tile 0, [128,256) S/P of tile 1,
-//               [256,256+d) PV of tile 0, [384,384+d) PV of tile 1.
-// P8 of tile t is written over the first 32 columns of its S region (4 e4m3 per
-// column); the MMA that overwrites them with the next S is issued after the PV
-// MMA that reads them, and tcgen05.mma ops of one thread execute in issue order.
+// CTA = one (sequence, query head, 128-row Q tile).  16 warps in four warpgroups,
+// registers traded with setmaxnreg (128 x 40 + 128 x 88 + 256 x 192 = 512 x 128,
+// the launch allocation):
+//   WG0  warp 0: TMA producer (Q once, K / V tiles into 3-stage rings)
+//        warp 1: TMEM owner and MMA issuer (one thread); warps 2-3 idle
+//          S(j)  = Q8 K8(j)^T   tcgen05.mma kind::i8 -> TMEM buffer j % 2 (double-buffered)
+//          PV(j) = P8(j) V8(j)  tcgen05.mma kind::f8f6f4, A = P8 from TMEM -> fresh FP32
+//   WG1  softmax for keys 0-63 of every KV tile   (one thread per query row)
+//   WG2  softmax for keys 64-127 of every KV tile (one thread per query row)
+//   WG3  two-level accumulation O = alpha O + PV(j) held in TMEM, and the epilogue
+// The two softmax warps of a lane quarter exchange their half-row maxima through
+// shared memory (one mbarrier per quarter and buffer), so both take the same running max.
 //
-// Per KV tile j the softmax thread of query row i (log2 domain, u = x * log2 e):
-//   u_j   = S_ij * (q_scale * k_scale_j * sm_scale * log2 e)   (S read as 12582912 + S)
+// TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256,256+d) PV(j),
+// [384,384+d) running O.  In S buffer b, P8 of keys 0-63 goes to columns 0-15 and
+// of keys 64-127 to columns 64-79 (4 e4m3 per column), each over columns its own
+// softmax warps have already read; the PV MMA takes one TMEM address per 32-key step.
+// Every S accumulates onto the magic pattern 0x4B400000 (fp32 1.5 * 2^23), so TMEM
+// returns bits(12582912 + S): softmax warps re-arm their columns after reading them,
+// the correction warps re-arm the P columns once PV has read them.
+//
+// Per KV tile j, query row i (log2 domain, u = x * log2 e):
+//   u_j   = S_ij * (q_scale * k_scale_j * sm_scale * log2 e)
 //   m'    = max(m, max_j u_j);  alpha = 2^(m - m')
 //   p_j   = 2^(u_j - m' + log2 448)   (= 448 * exp(x_j - x_max'), exp2_poly below)
 //   l     = l * alpha + sum_j p_j     (unquantized), P8_j = e4m3(p_j) -> TMEM
@@ -39,11 +44,13 @@
 
 namespace sage {
 
-constexpr int kAttnThreads = 384;
-constexpr int kAttnLaunchRegs = 168;  // 65536 / 384 rounded down to a multiple of 8
+constexpr int kAttnThreads = 512;
+constexpr int kAttnLaunchRegs = 128;  // 65536 / 512
 constexpr int kProducerRegs = 40;
-constexpr int kSoftmaxRegs = 232;
-static_assert(128 * kProducerRegs + 256 * kSoftmaxRegs <= kAttnThreads * kAttnLaunchRegs,
+constexpr int kCorrectionRegs = 88;
+constexpr int kSoftmaxRegs = 192;
+static_assert(128 * kProducerRegs + 128 * kCorrectionRegs + 256 * kSoftmaxRegs <=
+                  kAttnThreads * kAttnLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr int kKStages = 3;
 constexpr int kVStages = 3;
@@ -66,24 +73,22 @@ struct AttnArgs {
 
 template <int D>
 struct AttnSmem {
-  static constexpr int kTileQ = kBlkQ * D;      // bytes of one Q (or K) tile
-  static constexpr int kTileV = D * kKvTile;    // bytes of one V^T tile
+  static constexpr int kTileQ = kBlkQ * D;    // bytes of one Q (or K) tile
+  static constexpr int kTileV = D * kKvTile;  // bytes of one V^T tile
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + 2 * kTileQ;
+  static constexpr int kKOff = kQOff + kTileQ;
   static constexpr int kVOff = kKOff + kKStages * kTileQ;
-  static constexpr int kBarOff = kVOff + kVStages * kTileV;
-  // barriers: q_full, k_full[3], k_empty[3], v_full[3], v_empty[3], s_full[2], p_full[2],
-  // pv_full[2], mma_done, s_free[2]  -> 22 x 8 bytes, then the TMEM address slot
-  static constexpr int kNumBars = 22;
+  static constexpr int kXOff = kVOff + kVStages * kTileV;  // float xchg[2][2][128]
+  static constexpr int kAOff = kXOff + 2 * 2 * 128 * 4;    // float alpha[2][128]
+  static constexpr int kLOff = kAOff + 2 * 128 * 4;        // float lfin[2][128], mfin[128]
+  static constexpr int kBarOff = kLOff + 3 * 128 * 4;
+  // barriers: q_full, k_full[3], k_empty[3], v_full[3], v_empty[3], s_full[2], s_free[2],
+  // p_full[2], pv_full, pv_free, epi, mma_done, xchg[2][4] -> 31
+  static constexpr int kNumBars = 31;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kSlotOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
 };
-
-__device__ __forceinline__ float i2f_exact(uint32_t s) {
-  // exact int32 -> fp32 for |s| < 2^22: place s in the mantissa of 1.5 * 2^23
-  return __fsub_rn(__int_as_float(static_cast<int>(s) + 0x4B400000), 12582912.0f);
-}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -169,17 +174,6 @@ __device__ __forceinline__ f2 pair_of(const uint32_t (&r)[32], int k) {
 constexpr uint32_t kMagicBits = 0x4B400000u;
 constexpr float kMagic = 12582912.0f;
 
-// 32 lanes x 32 consecutive columns of TMEM all set to kMagicBits.
-__device__ __forceinline__ void tmem_fill_magic32(uint32_t taddr) {
-  const uint32_t v = kMagicBits;
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
-      "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
-      "r"(v)
-      : "memory");
-}
-
 // max over 32 magic-offset scores (masked entries hold 0, below every valid value)
 __device__ __forceinline__ float max32(const uint32_t (&r)[32], float acc) {
   float m0 = acc, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
@@ -244,7 +238,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
   constexpr uint32_t kSboQK = 8u * D;                  // 8 rows of D bytes
   constexpr uint32_t kIdescS = idesc_i8(128, kKvTile);
   constexpr uint32_t kIdescPV = idesc_e4m3_f32(128, D);
-  constexpr uint32_t kColS0 = 0, kColPV0 = 256;
+  constexpr uint32_t kColPV = 256, kColO = 384;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -256,28 +250,31 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
   auto bar_ke = [&](int s) { return bar0 + 8u * (4 + s); };
   auto bar_vf = [&](int s) { return bar0 + 8u * (7 + s); };
   auto bar_ve = [&](int s) { return bar0 + 8u * (10 + s); };
-  auto bar_s = [&](int t) { return bar0 + 8u * (13 + t); };
-  auto bar_p = [&](int t) { return bar0 + 8u * (15 + t); };
-  auto bar_pv = [&](int t) { return bar0 + 8u * (17 + t); };
-  const uint32_t bar_done = bar0 + 8u * 19;
-  auto bar_sf = [&](int t) { return bar0 + 8u * (20 + t); };
+  auto bar_sfull = [&](int b) { return bar0 + 8u * (13 + b); };
+  auto bar_sfree = [&](int b) { return bar0 + 8u * (15 + b); };
+  auto bar_pfull = [&](int b) { return bar0 + 8u * (17 + b); };
+  const uint32_t bar_pvfull = bar0 + 8u * 19;
+  const uint32_t bar_pvfree = bar0 + 8u * 20;
+  const uint32_t bar_epi = bar0 + 8u * 21;
+  const uint32_t bar_done = bar0 + 8u * 22;
+  // the two softmax warps of lane quarter q swap half-row maxima through xchg
+  auto bar_xchg = [&](int buf, int q) { return bar0 + 8u * (23 + 4 * buf + q); };
+  float* xchg = reinterpret_cast<float*>(smem + L::kXOff);  // [buffer][half][row]
+  float* alph = reinterpret_cast<float*>(smem + L::kAOff);  // [buffer][row]
+  float* lfin = reinterpret_cast<float*>(smem + L::kLOff);  // [half][row], then mfin[row]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wg = warp >> 2;
 
   // ---------------------------------------------------------------- work item
-  int b, hq, pair;
+  int b, hq, qt;
   {
     int idx = blockIdx.x;
+    int ntiles;
     if constexpr (std::is_same<Seq, SeqDense>::value) {
-      const int nq = (seq_len(seq, 0) + kBlkQ - 1) / kBlkQ;
-      const int pairs = (nq + 1) / 2;
-      const int g = idx % a.group; idx /= a.group;
-      pair = idx % pairs; idx /= pairs;
-      const int hk = idx % a.hkv;
-      b = idx / a.hkv;
-      hq = hk * a.group + g;
-      if (a.causal) pair = pairs - 1 - pair;  // heaviest pairs first
+      b = 0;
+      ntiles = (seq_len(seq, 0) + kBlkQ - 1) / kBlkQ;
     } else {
       int lo = 0, hi = seq.nseq - 1;
       while (lo < hi) {
@@ -287,39 +284,35 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       while (lo + 1 < seq.nseq && seq.cta[lo + 1] <= idx) ++lo;
       b = lo;
       idx -= seq.cta[b];
-      const int nq = (seq_len(seq, b) + kBlkQ - 1) / kBlkQ;
-      const int pairs = (nq + 1) / 2;
-      const int g = idx % a.group; idx /= a.group;
-      pair = idx % pairs; idx /= pairs;
-      hq = idx * a.group + g;
-      if (a.causal) pair = pairs - 1 - pair;
+      ntiles = (seq_len(seq, b) + kBlkQ - 1) / kBlkQ;
     }
+    const int g = idx % a.group; idx /= a.group;
+    qt = idx % ntiles; idx /= ntiles;
+    const int hk = idx % a.hkv;
+    if constexpr (std::is_same<Seq, SeqDense>::value) b = idx / a.hkv;
+    hq = hk * a.group + g;
+    if (a.causal) qt = ntiles - 1 - qt;  // longest rows first
   }
   const int hk = hq / a.group;
   const int n = seq_len(seq, b);
   const int off = seq_off(seq, b);
-  const int nq_tiles = (n + kBlkQ - 1) / kBlkQ;
-  const int nkv_all = (n + kKvTile - 1) / kKvTile;
-  int qt[2], nkv[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    qt[t] = 2 * pair + t;
-    nkv[t] = (qt[t] < nq_tiles) ? (a.causal ? qt[t] + 1 : nkv_all) : 0;
-  }
-  const int n_iter = max(nkv[0], nkv[1]);
+  const int nkv = a.causal ? qt + 1 : (n + kKvTile - 1) / kKvTile;
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     mbar_init(bar_q(), 1);
     for (int s = 0; s < kKStages; ++s) { mbar_init(bar_kf(s), 1); mbar_init(bar_ke(s), 1); }
     for (int s = 0; s < kVStages; ++s) { mbar_init(bar_vf(s), 1); mbar_init(bar_ve(s), 1); }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(bar_s(t), 1);
-      mbar_init(bar_p(t), 4);  // one arrival per softmax warp
-      mbar_init(bar_pv(t), 1);
-      mbar_init(bar_sf(t), 4);  // one arrival per softmax warp: S region re-armed
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_sfull(s), 1);
+      mbar_init(bar_sfree(s), 12);  // 8 softmax warps + 4 correction warps re-arm buffer s
+      mbar_init(bar_pfull(s), 8);   // 8 softmax warps wrote P (and alpha) into buffer s
     }
+    mbar_init(bar_pvfull, 1);
+    mbar_init(bar_pvfree, 4);
+    mbar_init(bar_epi, 8);
     mbar_init(bar_done, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bar_xchg(i >> 2, i & 3), 2);
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -337,20 +330,15 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
   const uint32_t tmem = *tmem_slot;
   const bool dead = watchdog_tripped();
 
-  if (warp < 4) {
+  if (wg == 0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
-   if (warp == 0) {
-    // ============================================================ TMA producer
-    if (lane == 0 && !dead) {
+    if (warp == 0 && lane == 0 && !dead) {
+      // ========================================================== TMA producer
       bool ok = true;
-      const int qbytes = (nkv[1] > 0 ? 2 : 1) * L::kTileQ;
-      mbar_arrive_expect_tx(bar_q(), qbytes);
-      for (int t = 0; t < 2; ++t)
-        if (nkv[t] > 0)
-          tma_load_2d(sbase + L::kQOff + t * L::kTileQ, &tmap_q, 0,
-                      hq * seq.t_pad + off + qt[t] * kBlkQ, bar_q());
+      mbar_arrive_expect_tx(bar_q(), L::kTileQ);
+      tma_load_2d(sbase + L::kQOff, &tmap_q, 0, hq * seq.t_pad + off + qt * kBlkQ, bar_q());
       int nk = 0, nv = 0;  // loads issued
-      for (int j = 0; j < n_iter && ok; ++j) {
+      for (int j = 0; j < nkv && ok; ++j) {
         const int ks = j % kKStages, vs = j % kVStages;
         if (j >= kKStages) ok = mbar_wait(bar_ke(ks), ((j / kKStages) - 1) & 1, 0x101);
         if (!ok) break;
@@ -374,246 +362,269 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       for (int jj = max(0, nv - kVStages); jj < nv; ++jj)
         while (!mbar_try_wait_sleep(bar_vf(jj % kVStages), (jj / kVStages) & 1) &&
                global_timer_ns() - t0 < kWaitLimitNs) {}
-    }
-  } else if (warp == 1) {
-    // ============================================================ MMA issuer
-    if (lane == 0 && !dead) {
-      // descriptors differ only in their start-address field (bits 0-13, address >> 4):
-      // keep one base per operand and add offsets at issue time
+    } else if (warp == 1 && lane == 0 && !dead) {
+      // ========================================================== MMA issuer
+      // descriptors differ only in their start-address field (bits 0-13, address >> 4)
       const uint64_t dq = sdesc_kmajor(sbase + L::kQOff, kSboQK, kSwizzle);
       const uint64_t dk = sdesc_kmajor(sbase + L::kKOff, kSboQK, kSwizzle);
       const uint64_t dv = sdesc_kmajor(sbase + L::kVOff, 1024u, 2u);
-      auto issue_s = [&](int t, int ks) {
-        const uint64_t aq = dq + static_cast<uint64_t>((t * L::kTileQ) >> 4);
+      auto issue_s = [&](int js) {  // S(js) = Q8 K8(js)^T onto the armed buffer js % 2
+        const int ks = js % kKStages;
         const uint64_t bk = dk + static_cast<uint64_t>((ks * L::kTileQ) >> 4);
-        const uint32_t d_tmem = tmem + kColS0 + 128u * t;
+        const uint32_t d_tmem = tmem + 128u * (js & 1);
 #pragma unroll
-        for (int s = 0; s < D / 32; ++s)
-          mma_i8_ss(d_tmem, aq + 2u * s, bk + 2u * s, kIdescS, 1u);
-        tc_commit(bar_s(t));
+        for (int s = 0; s < D / 32; ++s) mma_i8_ss(d_tmem, dq + 2u * s, bk + 2u * s, kIdescS, 1u);
+        tc_commit(bar_sfull(js & 1));
+        tc_commit(bar_ke(ks));
       };
-      auto issue_pv = [&](int t, int vs) {
+      auto issue_pv = [&](int j) {  // PV(j) = P8(j) V8(j) into a fresh FP32 accumulator
+        const int vs = j % kVStages;
         const uint64_t bv = dv + static_cast<uint64_t>((vs * L::kTileV) >> 4);
-        const uint32_t d_tmem = tmem + kColPV0 + 128u * t;
-        const uint32_t a_tmem = tmem + kColS0 + 128u * t;
+        const uint32_t p_tmem = tmem + 128u * (j & 1);
 #pragma unroll
-        for (int s = 0; s < kKvTile / 32; ++s)
-          mma_f8_ts(d_tmem, a_tmem + 8u * s, bv + 2u * s, kIdescPV, s > 0 ? 1u : 0u);
-        tc_commit(bar_pv(t));
+        for (int s = 0; s < kKvTile / 32; ++s) {
+          // keys 32s..32s+31: P8 columns 0, 8 (first half) and 64, 72 (second half)
+          const uint32_t a_col = (s < 2) ? 8u * s : 64u + 8u * (s - 2);
+          mma_f8_ts(tmem + kColPV, p_tmem + a_col, bv + 2u * s, kIdescPV, s > 0 ? 1u : 0u);
+        }
+        tc_commit(bar_pvfull);
+        tc_commit(bar_ve(vs));
       };
-      // S_t(j) accumulates onto the magic bit pattern the softmax warps wrote into the
-      // S region (re-armed after PV_t(j-1) consumed P_t(j-1)): wait for that first
-      bool ok = mbar_wait(bar_q(), 0, 0x201) && mbar_wait(bar_kf(0), 0, 0x202);
-      for (int t = 0; t < 2 && ok; ++t) {
-        if (nkv[t] == 0) continue;
-        ok = mbar_wait(bar_sf(t), 0, 0x207 + t);
+      bool ok = mbar_wait(bar_q(), 0, 0x201);
+      for (int js = 0; js < 2 && js < nkv && ok; ++js) {
+        ok = mbar_wait(bar_kf(js % kKStages), (js / kKStages) & 1, 0x202) &&
+             mbar_wait(bar_sfree(js & 1), 0, 0x203);
         if (!ok) break;
         tc_fence_after();
-        issue_s(t, 0);
+        issue_s(js);
       }
-      if (ok) tc_commit(bar_ke(0));
-      for (int j = 0; j < n_iter && ok; ++j) {
-        const int vs = j % kVStages;
-        bool v_ready = false, k_ready = false;
-        const int jn = j + 1, ksn = jn % kKStages;
-        bool issued_next = false;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j >= nkv[t]) continue;
-          ok = mbar_wait(bar_p(t), j & 1, 0x203 + t);
-          if (ok && !v_ready) { ok = mbar_wait(bar_vf(vs), (j / kVStages) & 1, 0x205); v_ready = true; }
+      for (int j = 0; j < nkv && ok; ++j) {
+        ok = mbar_wait(bar_pfull(j & 1), (j >> 1) & 1, 0x204) &&
+             mbar_wait(bar_vf(j % kVStages), (j / kVStages) & 1, 0x205) &&
+             (j == 0 || mbar_wait(bar_pvfree, (j - 1) & 1, 0x206));
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(j);
+        const int js = j + 2;
+        if (js < nkv) {
+          ok = mbar_wait(bar_kf(js % kKStages), (js / kKStages) & 1, 0x207) &&
+               mbar_wait(bar_sfree(js & 1), (js >> 1) & 1, 0x208);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(t, vs);
-          if (jn < nkv[t]) {
-            if (!k_ready) { ok = mbar_wait(bar_kf(ksn), (jn / kKStages) & 1, 0x206); k_ready = true; }
-            if (ok) ok = mbar_wait(bar_sf(t), jn & 1, 0x207 + t);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(t, ksn);
-            issued_next = true;
-          }
+          issue_s(js);
         }
-        if (!ok) break;
-        if (issued_next) tc_commit(bar_ke(ksn));
-        tc_commit(bar_ve(vs));
       }
       // every MMA issued by this thread has completed before TMEM is released
       tc_commit(bar_done);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait_sleep(bar_done, 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
     }
-   }
-  } else {
+  } else if (wg <= 2) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-    // ============================================================ softmax + correction
-    const int t = (warp - 4) >> 2;  // Q tile of this warpgroup
+    // ============================================================ softmax (one 64-key half)
+    const int h = wg - 1;           // 0: keys 0-63 of each KV tile, 1: keys 64-127
     const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
-    const int grow = qt[t] * kBlkQ + row;  // query index within the sequence
+    const int grow = qt * kBlkQ + row;  // query index within the sequence
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_base + kColS0 + 128u * t;
-    const uint32_t tPV = tmem + lane_base + kColPV0 + 128u * t;
-
-    f2 o2[D / 2];  // running output, columns (2c, 2c+1) in pair c
-#pragma unroll
-    for (int c = 0; c < D / 2; ++c) o2[c] = make_float2(0.0f, 0.0f);
-    float m = -INFINITY, l = 0.0f;
+    const uint32_t c0 = 64u * h;    // this half's S columns; its P8 takes the first 16
     bool ok = !dead;
-    const float sq = (nkv[t] > 0) ? a.q_scale[static_cast<int64_t>(hq) * (seq.t_pad / kBlkQ) +
-                                              off / kBlkQ + qt[t]]
-                                  : 0.0f;
+    const float sq = a.q_scale[static_cast<int64_t>(hq) * (seq.t_pad / kBlkQ) + off / kBlkQ + qt];
     const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kBlkK) + off / kBlkK;
 
-    // arm the S region: the first QK^T accumulates onto the magic bit pattern
-    if (ok && nkv[t] > 0) {
+    // arm this half's columns of both S buffers: the first two QK^T accumulate onto them
+    if (ok) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_fill_magic32(tS + 32u * c);
+      for (int buf = 0; buf < 2; ++buf) {
+        tmem_fill32(tmem + lane_base + 128u * buf + c0, kMagicBits);
+        tmem_fill32(tmem + lane_base + 128u * buf + c0 + 32u, kMagicBits);
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_sf(t));
+      if (lane == 0) { mbar_arrive(bar_sfree(0)); mbar_arrive(bar_sfree(1)); }
     }
 
-    for (int j = 0; j < nkv[t] && ok; ++j) {
+    float m = -INFINITY, l = 0.0f;
+    for (int j = 0; j < nkv && ok; ++j) {
+      const int buf = j & 1;
+      const uint32_t tS = tmem + lane_base + 128u * buf;
       const float ck0 = __fmul_rn(__fmul_rn(sq, ksc[2 * j]), a.scale_log2);
       const float ck1 = __fmul_rn(__fmul_rn(sq, ksc[2 * j + 1]), a.scale_log2);
-      const bool masked = (a.causal && j == qt[t]) || (j + 1) * kKvTile > n;
-      const int kv0 = j * kKvTile;
+      const float ck = h ? ck1 : ck0;
+      const bool masked = (a.causal && j == qt) || (j + 1) * kKvTile > n;
+      const int kv0 = j * kKvTile + 64 * h;  // first key of this half
       auto dropped = [&](int key) { return key >= n || (a.causal && key > grow); };
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_s(t), j & 1, 0x301 + t));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull(buf), (j >> 1) & 1, 0x301 + h));
       if (!ok) break;
       tc_fence_after();
 
-      // pass 1: largest score of each 64-key half (masked keys read as 0 < every valid value)
-      float hmax[2];
-      {
-        uint32_t ra[32], rb[32];
+      // pass 1: the largest magic-offset score of this half (masked keys read as 0,
+      // below every valid value 12582912 + S)
+      uint32_t ra[32], rb[32];
+      tmem_ld32(tS + c0, ra);
+      tmem_ld32(tS + c0 + 32u, rb);
+      tmem_wait_ld_tied(ra, rb);
+      uint32_t keep_a = 0xFFFFFFFFu, keep_b = 0xFFFFFFFFu;
+      if (masked) {
+        keep_a = 0u;
+        keep_b = 0u;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          tmem_ld32(tS + 64u * h, ra);
-          tmem_ld32(tS + 64u * h + 32u, rb);
-          tmem_wait_ld_tied(ra, rb);
-          if (masked) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              if (dropped(kv0 + 64 * h + i)) ra[i] = 0u;
-              if (dropped(kv0 + 64 * h + 32 + i)) rb[i] = 0u;
-            }
-          }
-          hmax[h] = max32(rb, max32(ra, 0.0f));
+        for (int i = 0; i < 32; ++i) {
+          if (dropped(kv0 + i)) ra[i] = 0u; else keep_a |= 1u << i;
+          if (dropped(kv0 + 32 + i)) rb[i] = 0u; else keep_b |= 1u << i;
         }
       }
-      // an all-masked half leaves 0; valid values are at least 12582912 - 2^21
-      const float mt = fmaxf(hmax[0] > 1.0e6f ? __fmul_rn(__fsub_rn(hmax[0], kMagic), ck0) : -INFINITY,
-                             hmax[1] > 1.0e6f ? __fmul_rn(__fsub_rn(hmax[1], kMagic), ck1) : -INFINITY);
+      const float hm = max32(rb, max32(ra, 0.0f));
+      // exchange half maxima with the other softmax warp of this lane quarter
+      xchg[(buf * 2 + h) * 128 + row] = hm;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_xchg(buf, quarter));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_xchg(buf, quarter), (j >> 1) & 1, 0x305 + h));
+      if (!ok) break;
+      const float ho = xchg[(buf * 2 + (1 - h)) * 128 + row];
+      const float hmax0 = h ? ho : hm, hmax1 = h ? hm : ho;
+      const float mt = fmaxf(hmax0 > 1.0e6f ? __fmul_rn(__fsub_rn(hmax0, kMagic), ck0) : -INFINITY,
+                             hmax1 > 1.0e6f ? __fmul_rn(__fsub_rn(hmax1, kMagic), ck1) : -INFINITY);
       const float m_new = fmaxf(m, mt);
       const float alpha = ex2(m - m_new);
       const float nbias = __fsub_rn(kLog2_448, m_new);
+      if (h == 0) alph[buf * 128 + row] = alpha;
 
-      // pass 2: p = 448 * 2^(u - m'), running sum, e4m3 P8 into TMEM columns 0-31,
-      // columns 32-127 re-armed with the magic pattern once read
+      // pass 2 on the same registers: p = 448 * 2^(u - m'), e4m3 P8 into this half's
+      // first 16 columns, the rest of the half re-armed with the magic pattern
       f2 acc = make_float2(0.0f, 0.0f);
-      {
-        uint32_t ra[32], rb[32];
-        uint32_t w[8];
-        auto finish = [&](uint32_t (&r)[32], int c) {
-          const float ck = c < 2 ? ck0 : ck1;
-          if (masked) {
-            uint32_t keep = 0u;
+      uint32_t w[8];
+      if (masked) p8_chunk<true>(ra, ck, nbias, acc, w, keep_a);
+      else p8_chunk<false>(ra, ck, nbias, acc, w, 0u);
+      tmem_st8(tS + c0, w);
+      if (masked) p8_chunk<true>(rb, ck, nbias, acc, w, keep_b);
+      else p8_chunk<false>(rb, ck, nbias, acc, w, 0u);
+      tmem_st8(tS + c0 + 8u, w);
+      tmem_fill16(tS + c0 + 16u, kMagicBits);
+      tmem_fill32(tS + c0 + 32u, kMagicBits);
+      l = l * alpha + (f2_lo(acc) + f2_hi(acc));
+      m = m_new;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) { mbar_arrive(bar_pfull(buf)); mbar_arrive(bar_sfree(buf)); }
+    }
+    // hand the row's partial sum (and, from the first half, its max) to the epilogue
+    lfin[h * 128 + row] = l;
+    if (h == 0) lfin[256 + row] = m;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_epi);
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCorrectionRegs));
+    // ============================================================ two-level accumulation
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int grow = qt * kBlkQ + row;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tPV = tmem + lane_base + kColPV;
+    const uint32_t tO = tmem + lane_base + kColO;
+    bool ok = !dead;
+
+    // arm the P8 columns (0-15 and 64-79) of both S buffers
+    if (ok) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) keep |= dropped(kv0 + 32 * c + i) ? 0u : (1u << i);
-            p8_chunk<true>(r, ck, nbias, acc, w, keep);
-          } else {
-            p8_chunk<false>(r, ck, nbias, acc, w, 0u);
-          }
-          tmem_st8(tS + 8u * c, w);
-          if (c > 0) tmem_fill_magic32(tS + 32u * c);
-        };
-        tmem_ld32(tS, ra);
-        tmem_wait_ld_tied(ra);
-        tmem_ld32(tS + 32u, rb);
-        finish(ra, 0);
-        tmem_wait_ld_tied(rb);
-        tmem_ld32(tS + 64u, ra);
-        finish(rb, 1);
-        tmem_wait_ld_tied(ra);
-        tmem_ld32(tS + 96u, rb);
-        finish(ra, 2);
-        tmem_wait_ld_tied(rb);
-        finish(rb, 3);
+      for (int buf = 0; buf < 2; ++buf) {
+        tmem_fill16(tmem + lane_base + 128u * buf, kMagicBits);
+        tmem_fill16(tmem + lane_base + 128u * buf + 64u, kMagicBits);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p(t));
-      l = l * alpha + (f2_lo(acc) + f2_hi(acc));
-      m = m_new;
+      if (lane == 0) { mbar_arrive(bar_sfree(0)); mbar_arrive(bar_sfree(1)); }
+    }
 
-      // two-level accumulation: O = alpha * O + PV_blk (PV_blk fresh in TMEM for this tile)
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_pv(t), j & 1, 0x303 + t));
+    for (int j = 0; j < nkv && ok; ++j) {
+      const int buf = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_pfull(buf), (j >> 1) & 1, 0x401)) &&
+           __all_sync(0xffffffffu, mbar_wait(bar_pvfull, j & 1, 0x402));
       if (!ok) break;
       tc_fence_after();
-      if (j + 1 < nkv[t]) {  // P consumed: re-arm columns 0-31 for the next QK^T
-        tmem_fill_magic32(tS);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_sf(t));
-      }
-      {
-        const f2 al = f2_make(alpha, alpha);
-        uint32_t ra[32], rb[32];
-        auto accum = [&](const uint32_t (&r)[32], int c) {
+      const f2 al = make_float2(alph[buf * 128 + row], alph[buf * 128 + row]);
+      // O = alpha * O + PV_blk, 32 columns at a time (the first tile just copies PV_blk)
 #pragma unroll
-          for (int i = 0; i < 16; ++i) o2[16 * c + i] = f2_fma(o2[16 * c + i], al, pair_of(r, i));
-        };
-        tmem_ld32(tPV, ra);
-        tmem_wait_ld_tied(ra);
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t rp[32], ro[32];
+        tmem_ld32(tPV + 32u * c, rp);
+        if (j > 0) {
+          tmem_ld32(tO + 32u * c, ro);
+          tmem_wait_ld_tied(rp, ro);
 #pragma unroll
-        for (int c = 0; c < D / 32; c += 2) {
-          tmem_ld32(tPV + 32u * (c + 1), rb);
-          accum(ra, c);
-          tmem_wait_ld_tied(rb);
-          if (c + 2 < D / 32) tmem_ld32(tPV + 32u * (c + 2), ra);
-          accum(rb, c + 1);
-          if (c + 2 < D / 32) tmem_wait_ld_tied(ra);
+          for (int i = 0; i < 16; ++i) {
+            const f2 o = f2_fma(pair_of(ro, i), al, pair_of(rp, i));
+            ro[2 * i] = __float_as_uint(o.x);
+            ro[2 * i + 1] = __float_as_uint(o.y);
+          }
+          tmem_st32(tO + 32u * c, ro);
+        } else {
+          tmem_wait_ld_tied(rp);
+          tmem_st32(tO + 32u * c, rp);
         }
       }
+      // PV_blk has been read: the next PV may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_pvfree);
+      // P8(j) has been consumed: re-arm its columns for S(j + 2)
+      tmem_fill16(tmem + lane_base + 128u * buf, kMagicBits);
+      tmem_fill16(tmem + lane_base + 128u * buf + 64u, kMagicBits);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_sfree(buf));
     }
 
     // ---------------------------------------------------------------- epilogue
-    if (ok && nkv[t] > 0 && grow < n) {
+    ok = ok && __all_sync(0xffffffffu, mbar_wait(bar_epi, 0, 0x403));
+    if (ok) {
+      tc_fence_after();
+      const float l = lfin[row] + lfin[128 + row];
+      const float m = lfin[256 + row];
       const float inv_l = 1.0f / l;
       const float* vs = a.v_scale + (static_cast<int64_t>(b) * a.hkv + hk) * D;
-      const int64_t orow = seq_base(seq, b, a.osb, a.ost) + hq * a.osh + static_cast<int64_t>(grow) * a.ost;
-      if (a.out_dtype == 2) {
-        float* dst = reinterpret_cast<float*>(a.out) + orow;
+      const int64_t orow =
+          seq_base(seq, b, a.osb, a.ost) + hq * a.osh + static_cast<int64_t>(grow) * a.ost;
 #pragma unroll
-        for (int c = 0; c < D; c += 4) {
-          float4 v = make_float4(f2_lo(o2[c / 2]) * vs[c] * inv_l, f2_hi(o2[c / 2]) * vs[c + 1] * inv_l,
-                                 f2_lo(o2[c / 2 + 1]) * vs[c + 2] * inv_l, f2_hi(o2[c / 2 + 1]) * vs[c + 3] * inv_l);
-          *reinterpret_cast<float4*>(dst + c) = v;
-        }
-      } else if (a.out_dtype == 1) {
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.out) + orow;
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ro[32];
+        tmem_ld32(tO + 32u * c, ro);
+        tmem_wait_ld_tied(ro);
+        if (grow < n) {
+          float v[32];
 #pragma unroll
-        for (int c = 0; c < D; c += 8) {
-          __align__(16) __nv_bfloat16 h8[8];
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ro[i]) * vs[32 * c + i] * inv_l;
+          if (a.out_dtype == 2) {
+            float* dst = reinterpret_cast<float*>(a.out) + orow + 32 * c;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) h8[i] = __float2bfloat16_rn(((i & 1) ? f2_hi(o2[(c + i) / 2]) : f2_lo(o2[(c + i) / 2])) * vs[c + i] * inv_l);
-          *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<const uint4*>(h8);
-        }
-      } else {
-        __half* dst = reinterpret_cast<__half*>(a.out) + orow;
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          } else if (a.out_dtype == 1) {
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.out) + orow + 32 * c;
 #pragma unroll
-        for (int c = 0; c < D; c += 8) {
-          __align__(16) __half h8[8];
+            for (int i = 0; i < 32; i += 8) {
+              __align__(16) __nv_bfloat16 h8[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) h8[i] = __float2half_rn(((i & 1) ? f2_hi(o2[(c + i) / 2]) : f2_lo(o2[(c + i) / 2])) * vs[c + i] * inv_l);
-          *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<const uint4*>(h8);
+              for (int e = 0; e < 8; ++e) h8[e] = __float2bfloat16_rn(v[i + e]);
+              *reinterpret_cast<uint4*>(dst + i) = *reinterpret_cast<const uint4*>(h8);
+            }
+          } else {
+            __half* dst = reinterpret_cast<__half*>(a.out) + orow + 32 * c;
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              __align__(16) __half h8[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) h8[e] = __float2half_rn(v[i + e]);
+              *reinterpret_cast<uint4*>(dst + i) = *reinterpret_cast<const uint4*>(h8);
+            }
+          }
         }
       }
-      if (a.lse != nullptr)
+      if (a.lse != nullptr && grow < n)
         a.lse[static_cast<int64_t>(hq) * seq.t_pad + off + grow] =
             m * 0.6931471805599453f + (logf(l) - kLn448);
     }

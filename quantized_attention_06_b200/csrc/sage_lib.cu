@@ -71,9 +71,9 @@ sage_status_t plan(const sage_problem_t* p, Layout& L, SeqVarlen* storage) {
         storage->cta[b] = static_cast<int32_t>(cta);
         if (b < p->batch) {
           const int n = cu[b + 1] - cu[b];
-          const int pairs = (n + 2 * kBlkQ - 1) / (2 * kBlkQ);
+          const int tiles = (n + kBlkQ - 1) / kBlkQ;  // one attention CTA per 128-row Q tile
           off += static_cast<int64_t>(round_up(n, kPad));
-          cta += static_cast<int64_t>(p->heads_q) * pairs;
+          cta += static_cast<int64_t>(p->heads_q) * tiles;
         }
       }
       L.var = storage;
@@ -333,8 +333,8 @@ sage_status_t sage_attn_fwd(const sage_problem_t* p, const int8_t* q8, const flo
     return d == 128 ? launch_attn<128>(*L.var, ncta, mq, mk, mv, a, s)
                     : launch_attn<64>(*L.var, ncta, mq, mk, mv, a, s);
   }
-  const int64_t pairs = (L.dense.len + 2 * kBlkQ - 1) / (2 * kBlkQ);
-  const int64_t ncta = static_cast<int64_t>(p->batch) * p->heads_q * pairs;
+  const int64_t tiles = (L.dense.len + kBlkQ - 1) / kBlkQ;
+  const int64_t ncta = static_cast<int64_t>(p->batch) * p->heads_q * tiles;
   return d == 128 ? launch_attn<128>(L.dense, ncta, mq, mk, mv, a, s)
                   : launch_attn<64>(L.dense, ncta, mq, mk, mv, a, s);
 }
