@@ -58,7 +58,8 @@ __all__ = [
     "k_channel_mean", "smooth_k", "quantize_int8_blocks", "quantize_v_e4m3",
     "integer_scores", "online_softmax_pv", "attention_head", "sage_attention",
     "reference_attention", "attention_weights",
-    "LOG2E_F32", "LOG2_448_F32", "EXP2_COEF_F32", "fma_f32", "exp2_f32", "kernel_scale_log2",
+    "LOG2E_F32", "LOG2_448_F32", "EXP2_COEF_F32", "EXP2_MAX_REL_ERR", "fma_f32", "exp2_f32",
+    "kernel_scale_log2",
     "online_softmax_pv_fp32_decision", "attention_head_kernel_precision",
 ]
 
@@ -352,8 +353,12 @@ def reference_attention(q, k, v, *, causal=False, sm_scale=None) -> np.ndarray:
 LOG2E_F32 = np.float32(1.4426950408889634)
 LOG2_448_F32 = np.float32(8.807354922057604)
 MAGIC_F32 = np.float32(12582912.0)           # 1.5 * 2^23
-EXP2_COEF_F32 = tuple(np.array([0x3F800000, 0x3F317AFE, 0x3E78062F, 0x3D6150BE],
+# 1 + c1 f + c2 f^2: minimal relative error for 2^f on [-1/2, 1/2] with the constant
+# term fixed at 1 (integer t then gives exact powers of two); max relative error
+# 1.97e-3, far below the e4m3 step of P (6.25% to 12.5%)
+EXP2_COEF_F32 = tuple(np.array([0x3F800000, 0x3F33F42F, 0x3E759F88],
                                dtype=np.uint32).view(np.float32))
+EXP2_MAX_REL_ERR = 1.97e-3
 
 
 def fma_f32(a, b, c) -> np.ndarray:
@@ -384,15 +389,14 @@ def fma_f32(a, b, c) -> np.ndarray:
 def exp2_f32(t) -> np.ndarray:
     """2^t in fp32 operations: r = t + 1.5*2^23 rounds t to n = rint(t) (magic-number
     rounding), f = t - (r - 1.5*2^23) in [-1/2, 1/2], Horner polynomial
-    1 + c1 f + c2 f^2 + c3 f^3 (fp32 FMAs), and n, clamped below at -125 so the
-    result stays a normal number, added to the exponent field."""
+    1 + c1 f + c2 f^2 (fp32 FMAs), and n, clamped below at -125 so the result
+    stays a normal number, added to the exponent field."""
     t = np.asarray(t, dtype=np.float32)
     r = (t + MAGIC_F32).astype(np.float32)
     n = np.maximum(r.view(np.int32), np.int32(0x4B400000 - 125)) - np.int32(0x4B400000)
     f = (t - (r - MAGIC_F32).astype(np.float32)).astype(np.float32)
-    c0, c1, c2, c3 = EXP2_COEF_F32
-    p = fma_f32(c3, f, c2)
-    p = fma_f32(p, f, c1)
+    c0, c1, c2 = EXP2_COEF_F32
+    p = fma_f32(c2, f, c1)
     p = fma_f32(p, f, c0)
     return (p.view(np.int32) + (n << 23)).view(np.float32)
 
@@ -446,12 +450,11 @@ def online_softmax_pv_fp32_decision(s_int, sq_rows, sk_blocks, scale_log2, valid
         tt = fma_f32(S.astype(np.float32), ckc, nbias[:, None])
         p = np.where(ok, exp2_f32(tt).astype(np.float64), 0.0)
         p8 = e4m3_round(p) if quantize_p else p
-        # fp64 accumulation in the frame of the fp32 running max (log2 domain)
+        # fp64 accumulation in the frame of the fp32 running max (log2 domain); the row
+        # sum takes the same unrounded p whose e4m3 codes feed PV, so the exp2
+        # approximation enters the numerator and the denominator alike
         alpha = np.where(np.isfinite(m32), np.exp2(m32.astype(np.float64) - m_new.astype(np.float64)), 0.0)
-        x_log2 = S * (sq_rows.astype(np.float64)[:, None] * skb[2 * j + half].astype(np.float64)[None, :]) \
-            * float(scale_log2)
-        e = np.where(ok, P_SCALE * np.exp2(x_log2 - m_new.astype(np.float64)[:, None]), 0.0)
-        l = l * alpha + np.sum(e, axis=1)
+        l = l * alpha + np.sum(p, axis=1)
         o = o * alpha[:, None] + p8 @ vvals[cols]
         m32 = m_new
     out = o * sv[None, :] / l[:, None]
@@ -464,7 +467,9 @@ def attention_head_kernel_precision(q, k, v, *, causal=False, sm_scale=None, row
     """attention_head with the P8 codes decided in the kernel's fp32 precision.
 
     Quantization of Q, K, V and the integer scores are the same exact stages as
-    attention_head; l, the rescale factors, PV and the output are fp64.
+    attention_head; p = 448 * 2^t comes from the fp32 logits and exp2 algorithm above,
+    P8 = e4m3(p), and the row sum l (of the unrounded p), the rescale factors, PV and
+    the output are fp64.
     """
     q = np.asarray(q, dtype=np.float32)
     k = np.asarray(k, dtype=np.float32)

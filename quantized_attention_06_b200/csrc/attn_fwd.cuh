@@ -25,8 +25,12 @@
 // of keys 64-127 to columns 64-79 (4 e4m3 per column), each over columns its own
 // softmax warps have already read; the PV MMA takes one TMEM address per 32-key step.
 // Every S accumulates onto the magic pattern 0x4B400000 (fp32 1.5 * 2^23), so TMEM
-// returns bits(12582912 + S): softmax warps re-arm their columns after reading them,
-// the correction warps re-arm the P columns once PV has read them.
+// returns bits(12582912 + S).  The pattern is written by the tensor core itself: before
+// the INT8 steps of S(j), one kind::f16 MMA with constant operands (every A entry 512,
+// every B entry 1536, K = 16, no accumulate) sets every element of the buffer to the
+// fp32 value 16 * 512 * 1536 = 12582912, and the INT8 steps add S onto those bits as
+// int32.  A buffer is free for S(j + 2) once the softmax warps have read S(j) and
+// written P8(j), and PV(j) has read P8(j).
 //
 // Per KV tile j, query row i (log2 domain, u = x * log2 e):
 //   u_j   = S_ij * (q_scale * k_scale_j * sm_scale * log2 e)
@@ -81,7 +85,11 @@ struct AttnSmem {
   static constexpr int kXOff = kVOff + kVStages * kTileV;  // float xchg[2][2][128]
   static constexpr int kAOff = kXOff + 2 * 2 * 128 * 4;    // float alpha[2][128]
   static constexpr int kLOff = kAOff + 2 * 128 * 4;        // float lfin[2][128], mfin[128]
-  static constexpr int kBarOff = kLOff + 3 * 128 * 4;
+  // constant f16 operands of the prefill MMA: 128 rows x 128 B each (128-byte swizzle
+  // atoms; every entry equal, so the layout is immaterial)
+  static constexpr int kCAOff = ((kLOff + 3 * 128 * 4) + 1023) / 1024 * 1024;
+  static constexpr int kCBOff = kCAOff + 128 * 128;
+  static constexpr int kBarOff = kCBOff + 128 * 128;
   // barriers: q_full, k_full[3], k_empty[3], v_full[3], v_empty[3], s_full[2], s_free[2],
   // p_full[2], pv_full, pv_free, epi, mma_done, xchg[2][4] -> 31
   static constexpr int kNumBars = 31;
@@ -99,19 +107,18 @@ __device__ __forceinline__ float ex2(float x) {
 // 2^t in plain IEEE fp32 operations, so that the P8 code it decides can be
 // reproduced exactly on any host: Cody-Waite split t = n + f with n = rint(t)
 // taken by magic-number rounding (r = t + 1.5 * 2^23, bits(r) = 0x4B400000 + n)
-// and f = t - (r - 1.5 * 2^23) in [-1/2, 1/2], a degree-3 polynomial for 2^f
+// and f = t - (r - 1.5 * 2^23) in [-1/2, 1/2], a degree-2 polynomial for 2^f
 // (coefficients fitted for minimal relative error with the constant term fixed at
-// 1; max relative error 1.0e-4), and n added to the exponent field, clamped below
-// at -125 so the result stays a normal number.
-constexpr float kExp2C1 = 0.693282962f;   // 0x3f317afe
-constexpr float kExp2C2 = 0.242211089f;   // 0x3e78062f
-constexpr float kExp2C3 = 0.0550086424f;  // 0x3d6150be
+// 1, so integer t gives exact powers of two; max relative error 1.97e-3, well below
+// the e4m3 step of P, which is 6.25% to 12.5%), and n added to the exponent field,
+// clamped below at -125 so the result stays a normal number.
+constexpr float kExp2C1 = 0.702944696f;  // 0x3f33f42f
+constexpr float kExp2C2 = 0.239866376f;  // 0x3e759f88
 constexpr int kExpClampBits = 0x4B400000 - 125;
 __device__ __forceinline__ float exp2_poly(float t) {
   const float r = __fadd_rn(t, 12582912.0f);
   const float f = __fsub_rn(t, __fsub_rn(r, 12582912.0f));
-  float p = __fmaf_rn(kExp2C3, f, kExp2C2);
-  p = __fmaf_rn(p, f, kExp2C1);
+  float p = __fmaf_rn(kExp2C2, f, kExp2C1);
   p = __fmaf_rn(p, f, 1.0f);
   const int rb = max(__float_as_int(r), kExpClampBits);
   return __int_as_float(__float_as_int(p) + rb * (1 << 23));
@@ -199,7 +206,6 @@ __device__ __forceinline__ void p8_chunk(const uint32_t (&r)[32], float ck, floa
   const f2 M = f2_make(kMagic, kMagic), NM = f2_make(-kMagic, -kMagic);
   const f2 NEG1 = f2_make(-1.0f, -1.0f), ONE = f2_make(1.0f, 1.0f);
   const f2 C1 = f2_make(kExp2C1, kExp2C1), C2 = f2_make(kExp2C2, kExp2C2);
-  const f2 C3 = f2_make(kExp2C3, kExp2C3);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     f2 pp[2];
@@ -208,8 +214,7 @@ __device__ __forceinline__ void p8_chunk(const uint32_t (&r)[32], float ck, floa
       const f2 t = f2_fma(f2_add(pair_of(r, 2 * i + h), NM), CK, NB);
       const f2 rr = f2_add(t, M);
       const f2 f = f2_fma(f2_add(rr, NM), NEG1, t);
-      f2 p = f2_fma(C3, f, C2);
-      p = f2_fma(p, f, C1);
+      f2 p = f2_fma(C2, f, C1);
       p = f2_fma(p, f, ONE);
       // bits(rr) = 0x4B400000 + n: max() clamps n at -125, and bits << 23 is n << 23
       // modulo 2^32
@@ -238,6 +243,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
   constexpr uint32_t kSboQK = 8u * D;                  // 8 rows of D bytes
   constexpr uint32_t kIdescS = idesc_i8(128, kKvTile);
   constexpr uint32_t kIdescPV = idesc_e4m3_f32(128, D);
+  constexpr uint32_t kIdescPre = idesc_f16_f32(128, kKvTile);
   constexpr uint32_t kColPV = 256, kColO = 384;
 
   extern __shared__ uint8_t smem_raw[];
@@ -324,6 +330,16 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
+  {
+    // prefill operands: f16 512.0 (0x6000) and 1536.0 (0x6600), two per word
+    uint32_t* ca = reinterpret_cast<uint32_t*>(smem + L::kCAOff);
+    uint32_t* cb = reinterpret_cast<uint32_t*>(smem + L::kCBOff);
+    for (int i = threadIdx.x; i < 128 * 128 / 4; i += kAttnThreads) {
+      ca[i] = 0x60006000u;
+      cb[i] = 0x66006600u;
+    }
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -340,13 +356,13 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       int nk = 0, nv = 0;  // loads issued
       for (int j = 0; j < nkv && ok; ++j) {
         const int ks = j % kKStages, vs = j % kVStages;
-        if (j >= kKStages) ok = mbar_wait(bar_ke(ks), ((j / kKStages) - 1) & 1, 0x101);
+        if (j >= kKStages) ok = mbar_wait<true>(bar_ke(ks), ((j / kKStages) - 1) & 1, 0x101);
         if (!ok) break;
         mbar_arrive_expect_tx(bar_kf(ks), L::kTileQ);
         tma_load_2d(sbase + L::kKOff + ks * L::kTileQ, &tmap_k, 0,
                     hk * seq.t_pad + off + j * kKvTile, bar_kf(ks));
         ++nk;
-        if (j >= kVStages) ok = mbar_wait(bar_ve(vs), ((j / kVStages) - 1) & 1, 0x102);
+        if (j >= kVStages) ok = mbar_wait<true>(bar_ve(vs), ((j / kVStages) - 1) & 1, 0x102);
         if (!ok) break;
         mbar_arrive_expect_tx(bar_vf(vs), L::kTileV);
         tma_load_2d(sbase + L::kVOff + vs * L::kTileV, &tmap_v, off + j * kKvTile, hk * D,
@@ -368,10 +384,14 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       const uint64_t dq = sdesc_kmajor(sbase + L::kQOff, kSboQK, kSwizzle);
       const uint64_t dk = sdesc_kmajor(sbase + L::kKOff, kSboQK, kSwizzle);
       const uint64_t dv = sdesc_kmajor(sbase + L::kVOff, 1024u, 2u);
+      const uint64_t dca = sdesc_kmajor(sbase + L::kCAOff, 1024u, 2u);
+      const uint64_t dcb = sdesc_kmajor(sbase + L::kCBOff, 1024u, 2u);
       auto issue_s = [&](int js) {  // S(js) = Q8 K8(js)^T onto the armed buffer js % 2
         const int ks = js % kKStages;
         const uint64_t bk = dk + static_cast<uint64_t>((ks * L::kTileQ) >> 4);
         const uint32_t d_tmem = tmem + 128u * (js & 1);
+#pragma unroll
+        mma_f16_ss(d_tmem, dca, dcb, kIdescPre, 0u);  // every element := 12582912.0f
 #pragma unroll
         for (int s = 0; s < D / 32; ++s) mma_i8_ss(d_tmem, dq + 2u * s, bk + 2u * s, kIdescS, 1u);
         tc_commit(bar_sfull(js & 1));
@@ -390,25 +410,25 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         tc_commit(bar_pvfull);
         tc_commit(bar_ve(vs));
       };
-      bool ok = mbar_wait(bar_q(), 0, 0x201);
+      bool ok = mbar_wait<true>(bar_q(), 0, 0x201);
       for (int js = 0; js < 2 && js < nkv && ok; ++js) {
-        ok = mbar_wait(bar_kf(js % kKStages), (js / kKStages) & 1, 0x202) &&
-             mbar_wait(bar_sfree(js & 1), 0, 0x203);
+        ok = mbar_wait<true>(bar_kf(js % kKStages), (js / kKStages) & 1, 0x202) &&
+             mbar_wait<true>(bar_sfree(js & 1), 0, 0x203);
         if (!ok) break;
         tc_fence_after();
         issue_s(js);
       }
       for (int j = 0; j < nkv && ok; ++j) {
-        ok = mbar_wait(bar_pfull(j & 1), (j >> 1) & 1, 0x204) &&
-             mbar_wait(bar_vf(j % kVStages), (j / kVStages) & 1, 0x205) &&
-             (j == 0 || mbar_wait(bar_pvfree, (j - 1) & 1, 0x206));
+        ok = mbar_wait<true>(bar_pfull(j & 1), (j >> 1) & 1, 0x204) &&
+             mbar_wait<true>(bar_vf(j % kVStages), (j / kVStages) & 1, 0x205) &&
+             (j == 0 || mbar_wait<true>(bar_pvfree, (j - 1) & 1, 0x206));
         if (!ok) break;
         tc_fence_after();
         issue_pv(j);
         const int js = j + 2;
         if (js < nkv) {
-          ok = mbar_wait(bar_kf(js % kKStages), (js / kKStages) & 1, 0x207) &&
-               mbar_wait(bar_sfree(js & 1), (js >> 1) & 1, 0x208);
+          ok = mbar_wait<true>(bar_kf(js % kKStages), (js / kKStages) & 1, 0x207) &&
+               mbar_wait<true>(bar_sfree(js & 1), (js >> 1) & 1, 0x208);
           if (!ok) break;
           tc_fence_after();
           issue_s(js);
@@ -432,18 +452,8 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const float sq = a.q_scale[static_cast<int64_t>(hq) * (seq.t_pad / kBlkQ) + off / kBlkQ + qt];
     const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kBlkK) + off / kBlkK;
 
-    // arm this half's columns of both S buffers: the first two QK^T accumulate onto them
-    if (ok) {
-#pragma unroll
-      for (int buf = 0; buf < 2; ++buf) {
-        tmem_fill32(tmem + lane_base + 128u * buf + c0, kMagicBits);
-        tmem_fill32(tmem + lane_base + 128u * buf + c0 + 32u, kMagicBits);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) { mbar_arrive(bar_sfree(0)); mbar_arrive(bar_sfree(1)); }
-    }
+    // both S buffers start free
+    if (ok && lane == 0) { mbar_arrive(bar_sfree(0)); mbar_arrive(bar_sfree(1)); }
 
     float m = -INFINITY, l = 0.0f;
     for (int j = 0; j < nkv && ok; ++j) {
@@ -492,7 +502,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       if (h == 0) alph[buf * 128 + row] = alpha;
 
       // pass 2 on the same registers: p = 448 * 2^(u - m'), e4m3 P8 into this half's
-      // first 16 columns, the rest of the half re-armed with the magic pattern
+      // first 16 columns
       f2 acc = make_float2(0.0f, 0.0f);
       uint32_t w[8];
       if (masked) p8_chunk<true>(ra, ck, nbias, acc, w, keep_a);
@@ -501,8 +511,6 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       if (masked) p8_chunk<true>(rb, ck, nbias, acc, w, keep_b);
       else p8_chunk<false>(rb, ck, nbias, acc, w, 0u);
       tmem_st8(tS + c0 + 8u, w);
-      tmem_fill16(tS + c0 + 16u, kMagicBits);
-      tmem_fill32(tS + c0 + 32u, kMagicBits);
       l = l * alpha + (f2_lo(acc) + f2_hi(acc));
       m = m_new;
       tmem_wait_st();
@@ -526,25 +534,17 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const uint32_t tO = tmem + lane_base + kColO;
     bool ok = !dead;
 
-    // arm the P8 columns (0-15 and 64-79) of both S buffers
-    if (ok) {
-#pragma unroll
-      for (int buf = 0; buf < 2; ++buf) {
-        tmem_fill16(tmem + lane_base + 128u * buf, kMagicBits);
-        tmem_fill16(tmem + lane_base + 128u * buf + 64u, kMagicBits);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) { mbar_arrive(bar_sfree(0)); mbar_arrive(bar_sfree(1)); }
-    }
+    // both S buffers start free
+    if (ok && lane == 0) { mbar_arrive(bar_sfree(0)); mbar_arrive(bar_sfree(1)); }
 
     for (int j = 0; j < nkv && ok; ++j) {
       const int buf = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_pfull(buf), (j >> 1) & 1, 0x401)) &&
-           __all_sync(0xffffffffu, mbar_wait(bar_pvfull, j & 1, 0x402));
+      ok = __all_sync(0xffffffffu, mbar_wait<true>(bar_pfull(buf), (j >> 1) & 1, 0x401)) &&
+           __all_sync(0xffffffffu, mbar_wait<true>(bar_pvfull, j & 1, 0x402));
       if (!ok) break;
       tc_fence_after();
+      // PV(j) has read P8(j): buffer j % 2 may take S(j + 2)
+      if (lane == 0) mbar_arrive(bar_sfree(buf));
       const f2 al = make_float2(alph[buf * 128 + row], alph[buf * 128 + row]);
       // O = alpha * O + PV_blk, 32 columns at a time (the first tile just copies PV_blk)
 #pragma unroll
@@ -566,17 +566,11 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
           tmem_st32(tO + 32u * c, rp);
         }
       }
-      // PV_blk has been read: the next PV may overwrite it
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_pvfree);
-      // P8(j) has been consumed: re-arm its columns for S(j + 2)
-      tmem_fill16(tmem + lane_base + 128u * buf, kMagicBits);
-      tmem_fill16(tmem + lane_base + 128u * buf + 64u, kMagicBits);
+      // PV_blk has been read and O written back: the next PV may overwrite PV_blk
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_sfree(buf));
+      if (lane == 0) mbar_arrive(bar_pvfree);
     }
 
     // ---------------------------------------------------------------- epilogue

@@ -81,8 +81,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // try_wait that may suspend the thread until the phase completes (or about
-// kSuspendHintNs elapses): used where a thread only drains before exiting.  The
-// hot-path waits below use the plain form, whose wake-up latency measured lower.
+// kSuspendHintNs elapses): the waiting warp leaves the scheduler instead of
+// polling, so it takes no issue slots from the warps it shares a scheduler with.
 constexpr uint32_t kSuspendHintNs = 0x989680u;  // 10 ms
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -97,16 +97,25 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 }
 
 // Wait for phase `parity` of an mbarrier, at most kWaitLimitNs.  On timeout the
-// watchdog word records `site` and false is returned; the caller must stop.
+// watchdog word records `site` and false is returned; the caller must stop.  The
+// poll loop is only try_wait; the watchdog word (a global load) and the clock are
+// looked at every kPollsPerCheck polls, so a completed phase is seen at once.
+// kSleep selects the suspending try_wait, for roles whose wake-up latency is hidden
+// (loads, MMA issue, accumulation): they then take no issue slots while they wait.
+constexpr uint32_t kPollsPerCheck = 256;
+template <bool kSleep = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto poll = [&]() { return kSleep ? mbar_try_wait_sleep(bar, parity) : mbar_try_wait(bar, parity); };
+  if (poll()) return true;
   const uint64_t t0 = global_timer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (watchdog_tripped()) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      watchdog_trip(site);
-      return false;
+  for (uint32_t it = 1;; ++it) {
+    if (poll()) return true;
+    if (kSleep || (it % kPollsPerCheck) == 0u) {
+      if (watchdog_tripped()) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        watchdog_trip(site);
+        return false;
+      }
     }
   }
 }
@@ -124,6 +133,20 @@ __device__ __forceinline__ bool elect_one() {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(pred));
   return pred != 0u;
+}
+
+// 16-byte shared-memory store.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// Make this thread's earlier shared-memory writes visible to the async proxy
+// (tensor-core operand reads) ordered after a following barrier arrive.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -187,6 +210,28 @@ __device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, f16 x f16 -> fp32 (both operands K-major).
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, e4m3 x e4m3 -> fp32 (both operands K-major).
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -283,6 +328,10 @@ __device__ __forceinline__ uint64_t sdesc_kmajor(uint32_t saddr, uint32_t sbo, u
 __host__ __device__ constexpr uint32_t idesc_i8(int m, int n) {
   return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(m >> 4) << 24);  // s32 <- s8 x s8
+}
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int m, int n) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(m >> 4) << 24);  // f32 <- f16 x f16
 }
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int m, int n) {
   return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |

@@ -405,7 +405,10 @@ def test_fma_f32_is_a_single_rounding():
 def test_exp2_f32_accuracy_and_exact_powers():
     t = np.linspace(-125, 9, 400001).astype(np.float32)
     p = orc.exp2_f32(t).astype(np.float64)
-    assert np.max(np.abs(p / np.exp2(t.astype(np.float64)) - 1)) <= 1.02e-4
+    err = np.max(np.abs(p / np.exp2(t.astype(np.float64)) - 1))
+    # the bound of the degree-2 polynomial on [-1/2, 1/2] (fp32 evaluation included),
+    # and not far below it: a dropped term or a wrong coefficient shows either way
+    assert 1.5e-3 <= err <= orc.EXP2_MAX_REL_ERR
     ti = np.arange(-125, 10).astype(np.float32)
     assert np.array_equal(orc.exp2_f32(ti), np.exp2(ti))
     assert np.all(np.diff(orc.exp2_f32(np.linspace(-3, 3, 10001).astype(np.float32))) >= 0)
@@ -417,7 +420,9 @@ def test_exp2_f32_accuracy_and_exact_powers():
 
 @pytest.mark.parametrize("causal", [False, True])
 def test_kernel_precision_path_without_p_rounding_is_softmax_attention(causal):
-    # with P left unrounded, the only approximation is the exp2 polynomial (1e-4)
+    # with P left unrounded, the only approximation is the exp2 polynomial: every
+    # weight is off by a factor 1 + e_i with |e_i| <= eps, which moves a normalized
+    # weighted mean of V by at most 2 eps max|V| and the log-sum by at most eps
     rng = np.random.default_rng(22)
     n, d = 333, 64
     q, k, v = (rng.standard_normal((n, d)).astype(np.float32) for _ in range(3))
@@ -430,22 +435,39 @@ def test_kernel_precision_path_without_p_rounding_is_softmax_attention(causal):
         x = np.where(np.arange(n)[None, :] > np.arange(n)[:, None], -np.inf, x)
     ref, lse = orc.online_softmax_pv(x, orc.e4m3_decode(r["v8"]), r["v_scale"].astype(np.float64),
                                      quantize_p=False)
-    scale = np.max(np.abs(ref))
-    assert np.max(np.abs(a["out"] - ref)) <= 3e-4 * scale
-    assert np.max(np.abs(a["lse"] - lse)) <= 1e-5
+    eps = orc.EXP2_MAX_REL_ERR
+    vmax = np.max(np.abs(orc.e4m3_decode(r["v8"]) * r["v_scale"].astype(np.float64)))
+    assert np.max(np.abs(a["out"] - ref)) <= 2.0 * eps / (1.0 - eps) * vmax
+    assert np.max(np.abs(a["lse"] - lse)) <= 1.01 * eps
 
 
-def test_kernel_precision_decision_matches_fp64_definition_closely():
+def test_kernel_precision_decision_is_as_accurate_as_fp64_decision():
+    # The kernel decides the P8 codes with fp32 arithmetic and a degree-2 exp2; the
+    # fp64 definition decides them from exact exponentials.  The two differ on a few
+    # percent of the codes (one e4m3 step each, see the test below), which on this
+    # short sequence moves single outputs by up to ~1e-2; measured against exact
+    # attention, both decisions are equally accurate, and the two outputs agree to
+    # cosine 0.9999.
     w = WORKLOADS["tiny"]
     x = generate(w)
+
+    def cos_l1(o, r):
+        o, r = o.ravel(), r.ravel()
+        return (float(o @ r / (np.linalg.norm(o) * np.linalg.norm(r))),
+                float(np.sum(np.abs(o - r)) / np.sum(np.abs(r))))
+
     for h in range(2):
-        a = orc.attention_head_kernel_precision(x["q"][0, h], x["k"][0, h], x["v"][0, h])
-        b = orc.attention_head(x["q"][0, h], x["k"][0, h], x["v"][0, h])
-        err = np.max(np.abs(a["out"] - b["out"]))
-        cos = float(a["out"].ravel() @ b["out"].ravel() /
-                    (np.linalg.norm(a["out"]) * np.linalg.norm(b["out"])))
-        assert cos >= 0.9999 and err <= 5e-3
-        assert np.max(np.abs(a["lse"] - b["lse"])) <= 1e-5
+        q, k, v = x["q"][0, h], x["k"][0, h], x["v"][0, h]
+        a = orc.attention_head_kernel_precision(q, k, v)
+        b = orc.attention_head(q, k, v)
+        ref = orc.reference_attention(q, k, v)
+        cos_a, l1_a = cos_l1(a["out"], ref)
+        cos_b, l1_b = cos_l1(b["out"], ref)
+        assert cos_a >= cos_b - 2e-5 and l1_a <= 1.05 * l1_b
+        assert cos_l1(a["out"], b["out"])[0] >= 0.9999
+        # the log-sum uses the unrounded p of each side: off by at most the
+        # polynomial's relative error
+        assert np.max(np.abs(a["lse"] - b["lse"])) <= 1.01 * orc.EXP2_MAX_REL_ERR
 
 
 def test_kernel_precision_p8_codes_mostly_equal_fp64_codes():
@@ -465,5 +487,12 @@ def test_kernel_precision_p8_codes_mostly_equal_fp64_codes():
     p32 = orc.e4m3_round(orc.exp2_f32(t).astype(np.float64))
     x = s * ck[None, :].astype(np.float64)
     p64 = orc.e4m3_round(448.0 * np.exp2(x - x.max(1, keepdims=True)))
-    assert np.mean(p32 == p64) >= 0.995
+    # a code differs only when p lies within the polynomial's relative error of an
+    # e4m3 rounding midpoint; midpoints sit at most 12.5% apart, so at most about
+    # 2 * eps / 0.0625 of the codes can move (6%), and most are far from a midpoint
+    same = np.mean(p32 == p64)
+    assert same >= 1.0 - 2.0 * orc.EXP2_MAX_REL_ERR / 0.0625
+    # and the codes that differ are neighbours
+    diff = p32 != p64
+    assert np.all(np.abs(np.log2(p32[diff] / p64[diff])) <= 0.19)
     del u
