@@ -257,9 +257,10 @@ def run_sage(args):
         e_steps = max(2, args.steps // 2)
 
         def e2e_step():
-            qd, kd, vd = (host[n].to(dev, non_blocking=True) for n in ("q", "k", "v"))
-            o = api.sageattn(qd, kd, vd, tensor_layout="HND", is_causal=args.causal)
-            host_out.copy_(o, non_blocking=True)
+            # the public host-buffer call: chunks of heads are copied in, quantized,
+            # attended and copied out, with the copies overlapping the kernels
+            api.sageattn_host(host["q"], host["k"], host["v"], tensor_layout="HND",
+                              is_causal=args.causal, out=host_out, synchronize=False)
 
         e2e_step()
         barrier()

@@ -18,8 +18,8 @@
  * ---------------------------------
  * - Pointers are device memory owned by the caller unless marked "host".  The
  *   library allocates no device memory and keeps no state between calls except
- *   the device watchdog word read by sage_poll_device_status() and the scratch
- *   array of sage_quant_qk_noalloc.
+ *   the device watchdog word read by sage_poll_device_status(), the scratch
+ *   array of sage_quant_qk_noalloc and the copy streams of sage_attn_host.
  * - Work is enqueued on `stream` (a cudaStream_t); calls return once enqueued.
  * - Errors: argument problems return SAGE_ERR_INVALID_ARGUMENT or
  *   SAGE_ERR_UNSUPPORTED before anything is enqueued; a failed launch returns
@@ -183,6 +183,39 @@ sage_status_t sage_attn_fwd(const sage_problem_t* p,
  */
 sage_status_t sage_debug_qk_int32(const sage_problem_t* p, const int8_t* q8, const int8_t* k8,
                                   int seq, int head_q, int32_t* s_out, sage_stream_t stream);
+
+/*
+ * sage_attn_host - the whole path (sage_quant_qk, sage_quant_v, sage_attn_fwd) on
+ * HOST buffers, pipelined over chunks of heads.  The pages describe no counterpart:
+ * it is the host-side driver of the calls above for inputs that live in host memory.
+ * Every head's quantization (mean, blocks, scales) and attention are independent of
+ * the other heads, so the outputs are bit-identical to the device path.
+ *   Dense problems only (cu_seqlens_host == NULL).  tensor_layout 0: q, k, v and out
+ *   are contiguous HND arrays (B, H, N, d); 1: contiguous NHD arrays (B, N, H, d).
+ *   q_host, k_host, v_host (dtype p->dtype) and out_host (out_dtype) are host memory;
+ *   page-locked memory lets the copies overlap the kernels (pageable memory works
+ *   but serializes).  Base pointers must be 16-byte aligned.
+ *   The KV heads of each batch entry are taken kv_heads_per_chunk at a time (with
+ *   their query heads); <= 0 picks a size giving at least 8 chunks.  For chunk c:
+ *   its inputs are copied in on an internal stream, its three kernel calls run on
+ *   `stream`, and its output is copied out on a second internal stream, so chunk c's
+ *   copy-in overlaps chunk c-1's kernels and chunk c-2's copy-out (two workspace
+ *   slots, one cudaMemcpyAsync or cudaMemcpy2DAsync per tensor and chunk).
+ *   `workspace` (device) must hold sage_host_workspace_bytes(p, kv_heads_per_chunk,
+ *   out_dtype) bytes.  The first copy waits for the work already on `stream`, and
+ *   `stream` waits for the last copy-out: synchronize `stream` before reading
+ *   out_host.  Calls on one device are serialized while they enqueue; the internal
+ *   streams and events are created on first use per device and kept.
+ * Errors as for the other entry points; SAGE_ERR_INVALID_ARGUMENT also for varlen
+ * problems, a bad layout code or a too-small workspace.
+ */
+size_t sage_host_workspace_bytes(const sage_problem_t* p, int kv_heads_per_chunk,
+                                 sage_dtype_t out_dtype);
+sage_status_t sage_attn_host(const sage_problem_t* p, int tensor_layout,
+                             const void* q_host, const void* k_host, const void* v_host,
+                             void* out_host, sage_dtype_t out_dtype, float sm_scale,
+                             int is_causal, int kv_heads_per_chunk, void* workspace,
+                             size_t workspace_bytes, sage_stream_t stream);
 
 /*
  * Synchronize `stream`, then read and clear the device watchdog word of the

@@ -23,7 +23,7 @@ SAGE_FP16, SAGE_BF16, SAGE_FP32 = 0, 1, 2
 EXPORTS = (
     "sage_buffer_sizes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd",
     "sage_debug_qk_int32", "sage_poll_device_status", "sage_quant_qk_noalloc",
-    "sage_status_string",
+    "sage_attn_host", "sage_host_workspace_bytes", "sage_status_string",
 )
 
 
@@ -74,10 +74,14 @@ def lib() -> ctypes.CDLL:
                                 ctypes.c_int, vp, ctypes.c_int, i64p, vp, vp]
     L.sage_debug_qk_int32.argtypes = [P(SageProblem), vp, vp, ctypes.c_int, ctypes.c_int, vp, vp]
     L.sage_poll_device_status.argtypes = [vp]
+    L.sage_attn_host.argtypes = [P(SageProblem), ctypes.c_int, vp, vp, vp, vp, ctypes.c_int,
+                                 ctypes.c_float, ctypes.c_int, ctypes.c_int, vp, sz, vp]
+    L.sage_host_workspace_bytes.argtypes = [P(SageProblem), ctypes.c_int, ctypes.c_int]
     L.sage_status_string.argtypes = [ctypes.c_int]
     L.sage_status_string.restype = ctypes.c_char_p
     for name in EXPORTS[:-1]:
         getattr(L, name).restype = ctypes.c_int
+    L.sage_host_workspace_bytes.restype = ctypes.c_size_t
     _lib = L
     return L
 

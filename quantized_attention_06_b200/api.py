@@ -23,7 +23,7 @@ import torch
 from . import _lib as L
 
 __all__ = ["Problem", "Quantized", "quant_qk", "quant_qk_noalloc", "quant_v", "attn_fwd",
-           "sageattn", "debug_qk_int32", "poll_device_status"]
+           "sageattn", "sageattn_host", "debug_qk_int32", "poll_device_status"]
 
 _IN_DTYPES = {torch.float16: L.SAGE_FP16, torch.bfloat16: L.SAGE_BF16}
 _OUT_DTYPES = {torch.float16: L.SAGE_FP16, torch.bfloat16: L.SAGE_BF16, torch.float32: L.SAGE_FP32}
@@ -218,6 +218,63 @@ def sageattn(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, cu_se
     quant_v(v, z)
     return attn_fwd(z, is_causal=is_causal, sm_scale=sm_scale, out_dtype=out_dtype,
                     return_lse=return_lse)
+
+
+_HOST_WS = {}
+
+
+def sageattn_host(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, out=None,
+                  out_dtype=None, kv_heads_per_chunk=0, device=None, synchronize=True):
+    """sageattn on host tensors (sage_attn_host): chunks of heads are copied in,
+    computed and copied out with the copies overlapping the kernels.
+
+    q, k, v: contiguous CPU tensors, (B, H, N, d) for "HND" or (B, N, H, d) for
+    "NHD", pinned for overlap.  Returns the output as a CPU tensor (pinned when
+    allocated here) of the same layout; with synchronize=False the call returns once
+    the work is enqueued on the current stream, and `out` must not be read before
+    that stream has been synchronized.
+    """
+    for t in (q, k, v):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("sageattn_host takes contiguous host tensors")
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if not torch.cuda.is_available():
+        raise RuntimeError("sageattn_host needs a CUDA device: there is no CPU fallback")
+    if tensor_layout == "HND":
+        b, hq, n, d = q.shape
+        hkv = k.shape[1]
+        code = 0
+    elif tensor_layout == "NHD":
+        b, n, hq, d = q.shape
+        hkv = k.shape[2]
+        code = 1
+    else:
+        raise ValueError(f"tensor_layout must be HND or NHD, got {tensor_layout}")
+    p = Problem(b, hq, hkv, n, d, q.dtype)
+    odt = out_dtype or q.dtype
+    if odt not in _OUT_DTYPES:
+        raise TypeError(f"unsupported output dtype {odt}")
+    if out is None:
+        out = torch.empty(q.shape, dtype=odt, pin_memory=True)
+    lib = L.lib()
+    need = int(lib.sage_host_workspace_bytes(ctypes.byref(p.c), int(kv_heads_per_chunk), _OUT_DTYPES[odt]))
+    if need == 0:
+        raise ValueError("sage_host_workspace_bytes rejected the problem")
+    key = (dev.index, need)
+    ws = _HOST_WS.get(key)
+    if ws is None:
+        _HOST_WS.clear()
+        ws = _HOST_WS[key] = torch.empty(need + 256, dtype=torch.uint8, device=dev)
+    base = (ws.data_ptr() + 255) // 256 * 256
+    with torch.cuda.device(dev):
+        st = lib.sage_attn_host(
+            ctypes.byref(p.c), code, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _OUT_DTYPES[odt],
+            ctypes.c_float(0.0 if sm_scale is None else float(sm_scale)), 1 if is_causal else 0,
+            int(kv_heads_per_chunk), ctypes.c_void_p(base), need, _stream())
+        L.check("sage_attn_host", st)
+        if synchronize:
+            torch.cuda.current_stream().synchronize()
+    return out
 
 
 def debug_qk_int32(z: Quantized, seq: int, head_q: int) -> torch.Tensor:

@@ -390,7 +390,6 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const int ks = js % kKStages;
         const uint64_t bk = dk + static_cast<uint64_t>((ks * L::kTileQ) >> 4);
         const uint32_t d_tmem = tmem + 128u * (js & 1);
-#pragma unroll
         mma_f16_ss(d_tmem, dca, dcb, kIdescPre, 0u);  // every element := 12582912.0f
 #pragma unroll
         for (int s = 0; s < D / 32; ++s) mma_i8_ss(d_tmem, dq + 2u * s, bk + 2u * s, kIdescS, 1u);

@@ -461,3 +461,217 @@ extern "C" sage_status_t sage_quant_qk_noalloc(const sage_problem_t* p, const vo
   }
 #undef SAGE_QK
 }
+
+// ---------------------------------------------------------------------------
+// sage_attn_host: the path on host buffers, pipelined over chunks of heads.
+// ---------------------------------------------------------------------------
+namespace {
+
+// Per device: the copy-in and copy-out streams and the events that order a chunk's
+// copy-in, kernels and copy-out across them (two workspace slots).
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t entry = nullptr, last = nullptr;
+  cudaEvent_t in_done[2] = {nullptr, nullptr}, k_done[2] = {nullptr, nullptr},
+              out_done[2] = {nullptr, nullptr};
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipe[kMaxDevices];
+
+sage_status_t pipe_for_device(HostPipe** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SAGE_ERR_CUDA;
+  HostPipe& P = g_pipe[dev];
+  if (!P.ready) {
+    const unsigned ef = cudaEventDisableTiming;
+    bool ok = cudaStreamCreateWithFlags(&P.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&P.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&P.entry, ef) == cudaSuccess &&
+              cudaEventCreateWithFlags(&P.last, ef) == cudaSuccess;
+    for (int i = 0; i < 2 && ok; ++i)
+      ok = cudaEventCreateWithFlags(&P.in_done[i], ef) == cudaSuccess &&
+           cudaEventCreateWithFlags(&P.k_done[i], ef) == cudaSuccess &&
+           cudaEventCreateWithFlags(&P.out_done[i], ef) == cudaSuccess;
+    if (!ok) return SAGE_ERR_CUDA;
+    P.ready = true;
+  }
+  *out = &P;
+  return SAGE_OK;
+}
+
+size_t dtype_bytes(sage_dtype_t t) { return t == SAGE_FP32 ? 4 : 2; }
+size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// The buffers of one workspace slot for a chunk problem of hc KV heads.
+struct Slot {
+  uint8_t *q, *k, *v, *out;
+  int8_t *q8, *k8;
+  float *q_scale, *k_scale, *k_mean, *v_scale;
+  uint8_t* v8;
+  void *ws_qk, *ws_v;
+  size_t ws_qk_bytes, ws_v_bytes, bytes;
+};
+
+// Lay out one slot from `base` (or only measure it when base is null).
+bool carve_slot(const sage_problem_t& cp, sage_dtype_t out_dtype, uint8_t* base, Slot* s) {
+  sage_sizes_t sz;
+  if (sage_buffer_sizes(&cp, &sz) != SAGE_OK) return false;
+  const size_t hd = static_cast<size_t>(cp.seqlen) * cp.head_dim;
+  const size_t in_q = static_cast<size_t>(cp.heads_q) * hd * 2, in_kv = static_cast<size_t>(cp.heads_kv) * hd * 2;
+  const size_t o = static_cast<size_t>(cp.heads_q) * hd * dtype_bytes(out_dtype);
+  size_t off = 0;
+  auto take = [&](size_t n) { uint8_t* ptr = base ? base + off : nullptr; off += up256(n); return ptr; };
+  s->q = take(in_q);
+  s->k = take(in_kv);
+  s->v = take(in_kv);
+  s->out = take(o);
+  s->q8 = reinterpret_cast<int8_t*>(take(sz.q8));
+  s->q_scale = reinterpret_cast<float*>(take(sz.q_scale));
+  s->k8 = reinterpret_cast<int8_t*>(take(sz.k8));
+  s->k_scale = reinterpret_cast<float*>(take(sz.k_scale));
+  s->k_mean = reinterpret_cast<float*>(take(sz.k_mean));
+  s->v8 = take(sz.v8);
+  s->v_scale = reinterpret_cast<float*>(take(sz.v_scale));
+  s->ws_qk = take(sz.workspace_qk);
+  s->ws_v = take(sz.workspace_v);
+  s->ws_qk_bytes = sz.workspace_qk;
+  s->ws_v_bytes = sz.workspace_v;
+  s->bytes = off;
+  return true;
+}
+
+int chunk_heads(const sage_problem_t* p, int kv_heads_per_chunk) {
+  int hc = kv_heads_per_chunk;
+  if (hc <= 0) {  // at least 8 chunks over the whole problem where the heads allow it
+    const int64_t units = static_cast<int64_t>(p->batch) * p->heads_kv;
+    hc = static_cast<int>(units / 8 < 1 ? 1 : units / 8);
+  }
+  return hc < p->heads_kv ? hc : p->heads_kv;
+}
+
+sage_problem_t chunk_problem(const sage_problem_t* p, int hc) {
+  sage_problem_t cp = *p;
+  const int g = p->heads_q / p->heads_kv;
+  cp.batch = 1;
+  cp.heads_kv = hc;
+  cp.heads_q = hc * g;
+  cp.cu_seqlens_host = nullptr;
+  return cp;
+}
+
+}  // namespace
+
+extern "C" size_t sage_host_workspace_bytes(const sage_problem_t* p, int kv_heads_per_chunk,
+                                            sage_dtype_t out_dtype) {
+  Layout L;
+  if (p == nullptr || p->cu_seqlens_host != nullptr || plan(p, L, nullptr) != SAGE_OK) return 0;
+  const sage_problem_t cp = chunk_problem(p, chunk_heads(p, kv_heads_per_chunk));
+  Slot s;
+  if (!carve_slot(cp, out_dtype, nullptr, &s)) return 0;
+  return 2 * s.bytes;
+}
+
+extern "C" sage_status_t sage_attn_host(const sage_problem_t* p, int tensor_layout,
+                                        const void* q_host, const void* k_host, const void* v_host,
+                                        void* out_host, sage_dtype_t out_dtype, float sm_scale,
+                                        int is_causal, int kv_heads_per_chunk, void* workspace,
+                                        size_t workspace_bytes, sage_stream_t stream) {
+  Layout L;
+  if (p == nullptr || p->cu_seqlens_host != nullptr) return SAGE_ERR_INVALID_ARGUMENT;
+  sage_status_t st = plan(p, L, nullptr);
+  if (st != SAGE_OK) return st;
+  if (tensor_layout != 0 && tensor_layout != 1) return SAGE_ERR_INVALID_ARGUMENT;
+  if (out_dtype != SAGE_FP16 && out_dtype != SAGE_BF16 && out_dtype != SAGE_FP32)
+    return SAGE_ERR_INVALID_ARGUMENT;
+  if (!q_host || !k_host || !v_host || !out_host || !workspace) return SAGE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q_host) || !aligned16(k_host) || !aligned16(v_host) || !aligned16(out_host) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return SAGE_ERR_INVALID_ARGUMENT;
+  const int hc = chunk_heads(p, kv_heads_per_chunk);
+  const sage_problem_t cfull = chunk_problem(p, hc);
+  Slot slot[2];
+  if (!carve_slot(cfull, out_dtype, nullptr, &slot[0])) return SAGE_ERR_INVALID_ARGUMENT;
+  if (workspace_bytes < 2 * slot[0].bytes) return SAGE_ERR_INVALID_ARGUMENT;
+  if ((st = device_ok()) != SAGE_OK) return st;
+
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe* P = nullptr;
+  if ((st = pipe_for_device(&P)) != SAGE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int g = p->heads_q / p->heads_kv;
+  const int64_t N = p->seqlen, d = p->head_dim;
+  const size_t ib = 2, ob = dtype_bytes(out_dtype);
+  // element strides {batch, head, token} of a chunk in its slot
+  auto slot_strides = [&](int heads, int64_t (&st3)[3]) {
+    if (tensor_layout == 0) { st3[0] = heads * N * d; st3[1] = N * d; st3[2] = d; }
+    else { st3[0] = N * heads * d; st3[1] = d; st3[2] = heads * d; }
+  };
+  // copy `heads` heads starting at head h0 of batch entry b between a host array of
+  // H heads and a contiguous slot buffer holding just those heads
+  auto copy = [&](void* dst, const void* src, int b, int h0, int heads, int H, size_t eb, bool to_dev,
+                  cudaStream_t cs) -> bool {
+    const size_t row = static_cast<size_t>(d) * eb;  // one (token, head) row
+    if (tensor_layout == 0) {
+      const size_t host_off = (static_cast<size_t>(b) * H + h0) * N * row;
+      const size_t n = static_cast<size_t>(heads) * N * row;
+      return to_dev ? cudaMemcpyAsync(dst, static_cast<const uint8_t*>(src) + host_off, n,
+                                      cudaMemcpyHostToDevice, cs) == cudaSuccess
+                    : cudaMemcpyAsync(static_cast<uint8_t*>(dst) + host_off, src, n,
+                                      cudaMemcpyDeviceToHost, cs) == cudaSuccess;
+    }
+    const size_t host_off = static_cast<size_t>(b) * N * H * row + h0 * row;
+    const size_t hpitch = H * row, dpitch = heads * row, width = heads * row;
+    return to_dev ? cudaMemcpy2DAsync(dst, dpitch, static_cast<const uint8_t*>(src) + host_off, hpitch,
+                                      width, N, cudaMemcpyHostToDevice, cs) == cudaSuccess
+                  : cudaMemcpy2DAsync(static_cast<uint8_t*>(dst) + host_off, hpitch, src, dpitch,
+                                      width, N, cudaMemcpyDeviceToHost, cs) == cudaSuccess;
+  };
+
+  // the slots' previous users are the work already enqueued on `stream`
+  if (cudaEventRecord(P->entry, s) != cudaSuccess ||
+      cudaStreamWaitEvent(P->h2d, P->entry, 0) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  int c = 0;
+  for (int b = 0; b < p->batch; ++b) {
+    for (int h0 = 0; h0 < p->heads_kv; h0 += hc, ++c) {
+      const int heads = (p->heads_kv - h0 < hc) ? p->heads_kv - h0 : hc;
+      const sage_problem_t cp = chunk_problem(p, heads);
+      const int i = c & 1;
+      carve_slot(cp, out_dtype, static_cast<uint8_t*>(workspace) + i * slot[0].bytes, &slot[i]);
+      Slot& S = slot[i];
+      // copy-in: the slot's inputs are free once chunk c-2's kernels are done
+      if (c >= 2 && cudaStreamWaitEvent(P->h2d, P->k_done[i], 0) != cudaSuccess) return SAGE_ERR_CUDA;
+      if (!copy(S.q, q_host, b, h0 * g, heads * g, p->heads_q, ib, true, P->h2d) ||
+          !copy(S.k, k_host, b, h0, heads, p->heads_kv, ib, true, P->h2d) ||
+          !copy(S.v, v_host, b, h0, heads, p->heads_kv, ib, true, P->h2d) ||
+          cudaEventRecord(P->in_done[i], P->h2d) != cudaSuccess)
+        return SAGE_ERR_CUDA;
+      // kernels on `stream`: after the copy-in, and after chunk c-2's copy-out has
+      // read this slot's output buffer
+      if (cudaStreamWaitEvent(s, P->in_done[i], 0) != cudaSuccess) return SAGE_ERR_CUDA;
+      if (c >= 2 && cudaStreamWaitEvent(s, P->out_done[i], 0) != cudaSuccess) return SAGE_ERR_CUDA;
+      int64_t qs[3], ks[3];
+      slot_strides(heads * g, qs);
+      slot_strides(heads, ks);
+      if ((st = sage_quant_qk(&cp, S.q, qs, S.k, ks, S.q8, S.q_scale, S.k8, S.k_scale, S.k_mean,
+                              S.ws_qk, S.ws_qk_bytes, stream)) != SAGE_OK)
+        return st;
+      if ((st = sage_quant_v(&cp, S.v, ks, S.v8, S.v_scale, S.ws_v, S.ws_v_bytes, stream)) != SAGE_OK)
+        return st;
+      if ((st = sage_attn_fwd(&cp, S.q8, S.q_scale, S.k8, S.k_scale, S.v8, S.v_scale, sm_scale,
+                              is_causal, S.out, out_dtype, qs, nullptr, stream)) != SAGE_OK)
+        return st;
+      if (cudaEventRecord(P->k_done[i], s) != cudaSuccess) return SAGE_ERR_CUDA;
+      // copy-out
+      if (cudaStreamWaitEvent(P->d2h, P->k_done[i], 0) != cudaSuccess ||
+          !copy(out_host, S.out, b, h0 * g, heads * g, p->heads_q, ob, false, P->d2h) ||
+          cudaEventRecord(P->out_done[i], P->d2h) != cudaSuccess)
+        return SAGE_ERR_CUDA;
+    }
+  }
+  // `stream` continues after the last copy-out
+  if (cudaEventRecord(P->last, P->d2h) != cudaSuccess || cudaStreamWaitEvent(s, P->last, 0) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  return SAGE_OK;
+}

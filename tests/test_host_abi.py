@@ -23,7 +23,7 @@ def lib():
 
 def _declared_symbols():
     src = open(os.path.join(ROOT, "include", "sage.h")).read()
-    return sorted(set(re.findall(r"^\s*(?:sage_status_t|const char\*)\s+(sage_\w+)\(", src, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:sage_status_t|const char\*|size_t)\s+(sage_\w+)\(", src, re.M)))
 
 
 def test_exports_every_declared_symbol(lib):
@@ -118,3 +118,41 @@ def test_valid_call_without_gpu_fails_loudly(lib):
         api.sageattn(torch.zeros(1, 2, 256, 64, dtype=torch.float16),
                      torch.zeros(1, 2, 256, 64, dtype=torch.float16),
                      torch.zeros(1, 2, 256, 64, dtype=torch.float16))  # ... compute does not
+
+
+def _attn_host(lib, p, layout=0, ptr=FAKE, ws=FAKE, ws_bytes=1 << 40, chunk=0, odt=L.SAGE_FP16):
+    return lib.sage_attn_host(ctypes.byref(p), layout, ptr, FAKE, FAKE, FAKE, odt, ctypes.c_float(0.0),
+                              0, chunk, ws, ws_bytes, None)
+
+
+def test_host_pipeline_workspace_and_validation(lib):
+    p = _problem(b=2, hq=4, hkv=2, n=300, d=128)
+    # default chunking: at least 8 chunks where possible -> one KV head per chunk here
+    one = lib.sage_host_workspace_bytes(ctypes.byref(p), 1, L.SAGE_FP16)
+    assert one > 0 and lib.sage_host_workspace_bytes(ctypes.byref(p), 0, L.SAGE_FP16) == one
+    two = lib.sage_host_workspace_bytes(ctypes.byref(p), 2, L.SAGE_FP16)
+    assert two > one
+    # a slot holds q, k, v and the output of its heads plus the quantized buffers
+    st, s = _sizes(lib, _problem(b=1, hq=2, hkv=1, n=300, d=128))
+    assert st == 0
+    q_in, kv_in, o = 2 * 300 * 128 * 2, 300 * 128 * 2, 2 * 300 * 128 * 2
+    parts = [q_in, kv_in, kv_in, o, s.q8, s.q_scale, s.k8, s.k_scale, s.k_mean, s.v8, s.v_scale,
+             s.workspace_qk, s.workspace_v]
+    assert one == 2 * sum((x + 255) // 256 * 256 for x in parts)
+    assert lib.sage_host_workspace_bytes(ctypes.byref(p), 1, L.SAGE_FP32) > one
+    # rejected before anything is enqueued
+    assert _attn_host(lib, p, layout=2) == L.SAGE_ERR_INVALID_ARGUMENT
+    assert _attn_host(lib, p, ptr=None) == L.SAGE_ERR_INVALID_ARGUMENT
+    assert _attn_host(lib, p, ptr=FAKE + 8) == L.SAGE_ERR_INVALID_ARGUMENT
+    assert _attn_host(lib, p, ws=FAKE + 16) == L.SAGE_ERR_INVALID_ARGUMENT      # slots are 256-aligned
+    assert _attn_host(lib, p, chunk=1, ws_bytes=one - 1) == L.SAGE_ERR_INVALID_ARGUMENT
+    assert _attn_host(lib, p, odt=7) == L.SAGE_ERR_INVALID_ARGUMENT
+    vl = _problem(hq=4, hkv=2, d=128, cu=[0, 100, 300])
+    assert lib.sage_host_workspace_bytes(ctypes.byref(vl), 0, L.SAGE_FP16) == 0
+    assert _attn_host(lib, vl) == L.SAGE_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the GPU-less host")
+def test_host_pipeline_without_gpu_fails_loudly(lib):
+    p = _problem(b=1, hq=2, hkv=2, n=256, d=64)
+    assert _attn_host(lib, p) == L.SAGE_ERR_CUDA
