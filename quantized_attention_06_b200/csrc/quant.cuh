@@ -254,44 +254,70 @@ struct VQuantArgs {
 template <typename T, int D, class Seq>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_v_kernel(const __grid_constant__ Seq seq, const __grid_constant__ VQuantArgs a) {
-  constexpr int VPR = D / 8;
-  constexpr int RG = kQuantThreads / VPR;
-  constexpr int IT = kPad / RG;
-  constexpr int LD = kPad + 16;  // padded smem row (bytes) of the transposed tile
-  __shared__ __align__(16) uint8_t tile[D][LD];
+  // One CTA: one 128-token block of one KV head.  Thread (cg, tg) converts channels
+  // 8cg .. 8cg+7 of tokens TPT*tg .. TPT*tg+TPT-1, pairing two tokens of one channel
+  // per e4m3x2 conversion, so each channel's TPT codes leave the thread as one
+  // TPT-byte word.  The words go into a [D][128] byte tile whose 16-byte chunks are
+  // XOR-swizzled by (channel % 8), and each channel row then leaves as 16-byte
+  // stores of the token-contiguous output.
+  constexpr int CG = D / 8;                  // channel groups (16-byte input vectors)
+  constexpr int TG = kQuantThreads / CG;     // token groups
+  constexpr int TPT = kPad / TG;             // tokens per thread: 8 (d = 128) or 4 (d = 64)
+  static_assert(TPT == 4 || TPT == 8, "tile shape");
+  __shared__ __align__(16) uint8_t tile[D * kPad];
   const int pb = blockIdx.x, h = blockIdx.y;
   const SeqPos sp = locate(seq, pb * kPad, a.sb, a.st);
   const int t0 = pb * kPad - sp.off;
-  const int vc = threadIdx.x % VPR, rg = threadIdx.x / VPR;
-  const T* src = reinterpret_cast<const T*>(a.v) + sp.base + h * a.sh + vc * 8;
+  const int cg = threadIdx.x % CG, tg = threadIdx.x / CG;
+  const T* src = reinterpret_cast<const T*>(a.v) + sp.base + h * a.sh + cg * 8;
   float r[8];
   {
-    const float* vm = a.vmax + (static_cast<int64_t>(sp.b) * a.hkv + h) * D + vc * 8;
+    const float* vm = a.vmax + (static_cast<int64_t>(sp.b) * a.hkv + h) * D + cg * 8;
 #pragma unroll
     for (int i = 0; i < 8; ++i) r[i] = (vm[i] > 0.0f) ? __fdiv_rn(448.0f, vm[i]) : 0.0f;
   }
+  // codes[c][u]: e4m3 of channel 8cg+c for tokens (2u, 2u+1) of this thread, 16 bits
+  uint32_t codes[8][TPT / 2];
 #pragma unroll
-  for (int it = 0; it < IT; ++it) {
-    const int rr = rg + it * RG;
-    const int t = t0 + rr;
-    const bool valid = t < sp.n;
-    const uint4 v = valid ? ld_stream16(src + t * a.st) : make_uint4(0, 0, 0, 0);
-    float f[8];
-    unpack8<T>(v, f);
+  for (int u = 0; u < TPT / 2; ++u) {
+    const int ta = t0 + TPT * tg + 2 * u, tb = ta + 1;
+    const bool va = ta < sp.n, vb = tb < sp.n;
+    float fa[8], fb[8];
+    unpack8<T>(va ? ld_stream16(src + static_cast<int64_t>(ta) * a.st) : make_uint4(0, 0, 0, 0), fa);
+    unpack8<T>(vb ? ld_stream16(src + static_cast<int64_t>(tb) * a.st) : make_uint4(0, 0, 0, 0), fb);
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      const uint32_t two = valid ? e4m3x2(__fmul_rn(f[i], r[i]), __fmul_rn(f[i + 1], r[i + 1])) : 0u;
-      tile[vc * 8 + i][rr] = static_cast<uint8_t>(two & 0xFFu);
-      tile[vc * 8 + i + 1][rr] = static_cast<uint8_t>(two >> 8);
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t two = e4m3x2(__fmul_rn(fa[c], r[c]), __fmul_rn(fb[c], r[c]));
+      codes[c][u] = two & ((va ? 0xFFu : 0u) | (vb ? 0xFF00u : 0u));  // padding tokens: 0
     }
+  }
+  // channel order rotated by cg: lanes cg and cg + 8 share a bank, no more
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int c = (k + cg) & 7;
+    const int ch = cg * 8 + c;
+    const int tok = TPT * tg;  // first token of this thread within the block
+    const int off = ch * kPad + ((((tok >> 4) ^ ch) & 7) << 4) + (tok & 15);
+    uint32_t w0 = 0u, w1 = 0u;
+#pragma unroll
+    for (int u = 0; u < TPT / 2; ++u) {
+      // select this channel's codes without a dynamically indexed register array
+      uint32_t v = 0u;
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) v = (cc == c) ? codes[cc][u] : v;
+      if (u < 2) w0 |= v << (16 * u);
+      else w1 |= v << (16 * (u - 2));
+    }
+    if (TPT == 8) *reinterpret_cast<uint2*>(tile + off) = make_uint2(w0, w1);
+    else *reinterpret_cast<uint32_t*>(tile + off) = w0;
   }
   __syncthreads();
   // each channel row of the tile is 128 contiguous output bytes: 8 threads x 16 B
   uint8_t* dst = a.v8 + static_cast<int64_t>(h) * D * seq.t_pad + pb * kPad;
   for (int i = threadIdx.x; i < D * 8; i += kQuantThreads) {
-    const int c = i >> 3, j = i & 7;
-    const uint4 w = *reinterpret_cast<const uint4*>(&tile[c][j * 16]);
-    *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(c) * seq.t_pad + j * 16) = w;
+    const int ch = i >> 3, j = i & 7;
+    const uint4 w = *reinterpret_cast<const uint4*>(tile + ch * kPad + ((j ^ (ch & 7)) << 4));
+    *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(ch) * seq.t_pad + j * 16) = w;
   }
 }
 
