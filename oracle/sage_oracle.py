@@ -230,13 +230,16 @@ def online_softmax_pv(x_rows: np.ndarray, vvals: np.ndarray, sv: np.ndarray,
 
 
 def attention_head(q, k, v, *, causal: bool = False, sm_scale: float | None = None,
-                   rows=None, quantize: bool = True, smooth: bool = True) -> dict:
+                   rows=None, quantize: bool = True, smooth: bool = True,
+                   qblk: int = BLKQ, kblk: int = BLKK) -> dict:
     """Quantized attention for one (sequence, query head) with its KV head.
 
     q: (n, d), k, v: (n_kv, d), float32 holding the input values.  ``rows`` picks a
     subset of query rows (all by default); every row is computed independently.
     ``quantize=False`` replaces every quantizer by the identity (fp64 values,
-    P unrounded), which reduces the method to exact softmax attention.
+    P unrounded), which reduces the method to exact softmax attention.  qblk / kblk
+    are the INT8 scale blocks of Q and K in tokens (128 / 64 as the method states;
+    1 / 32 for the per-thread granularity).
     """
     q = np.asarray(q, dtype=np.float32)
     k = np.asarray(k, dtype=np.float32)
@@ -252,12 +255,12 @@ def attention_head(q, k, v, *, causal: bool = False, sm_scale: float | None = No
     res = {"k_mean": mu}
     if quantize:
         ks = smooth_k(k, mu)
-        q8, sq = quantize_int8_blocks(q, BLKQ)
-        k8, sk = quantize_int8_blocks(ks, BLKK)
+        q8, sq = quantize_int8_blocks(q, qblk)
+        k8, sk = quantize_int8_blocks(ks, kblk)
         v8, sv = quantize_v_e4m3(v)
         s_int = integer_scores(q8[rows], k8[:n_kv])
-        row_scale = sq[rows // BLKQ].astype(np.float64)
-        col_scale = sk[np.arange(n_kv) // BLKK].astype(np.float64)
+        row_scale = sq[rows // qblk].astype(np.float64)
+        col_scale = sk[np.arange(n_kv) // kblk].astype(np.float64)
         x = s_int.astype(np.float64) * row_scale[:, None] * col_scale[None, :] * scale
         vvals = e4m3_decode(v8)
         svv = sv.astype(np.float64)
@@ -300,7 +303,7 @@ def attention_weights(q, k, *, causal=False, sm_scale=None, quantize=True, smoot
 
 
 def sage_attention(q, k, v, *, causal=False, sm_scale=None, cu_seqlens=None,
-                   quantize=True, smooth=True) -> np.ndarray:
+                   quantize=True, smooth=True, qblk: int = BLKQ, kblk: int = BLKK) -> np.ndarray:
     """Whole-batch quantized attention in float64.
 
     Dense: q (B,Hq,N,d), k, v (B,Hkv,N,d) -> out (B,Hq,N,d).
@@ -314,7 +317,7 @@ def sage_attention(q, k, v, *, causal=False, sm_scale=None, cu_seqlens=None,
             for h in range(Hq):
                 out[b, h] = attention_head(q[b, h], k[b, h // g], v[b, h // g], causal=causal,
                                            sm_scale=sm_scale, quantize=quantize,
-                                           smooth=smooth)["out"]
+                                           smooth=smooth, qblk=qblk, kblk=kblk)["out"]
         return out
     T, Hq, d = q.shape
     g = Hq // k.shape[1]
@@ -323,7 +326,7 @@ def sage_attention(q, k, v, *, causal=False, sm_scale=None, cu_seqlens=None,
         for h in range(Hq):
             out[s0:s1, h] = attention_head(q[s0:s1, h], k[s0:s1, h // g], v[s0:s1, h // g],
                                            causal=causal, sm_scale=sm_scale, quantize=quantize,
-                                           smooth=smooth)["out"]
+                                           smooth=smooth, qblk=qblk, kblk=kblk)["out"]
     return out
 
 
@@ -408,19 +411,20 @@ def kernel_scale_log2(d: int, sm_scale: float | None = None) -> np.float32:
 
 
 def online_softmax_pv_fp32_decision(s_int, sq_rows, sk_blocks, scale_log2, valid, vvals, sv,
-                                    quantize_p: bool = True):
+                                    quantize_p: bool = True, kblk: int = BLKK):
     """Online softmax with the P8 codes decided in the kernel's fp32 precision.
 
     s_int: (r, n_kv) exact scores; sq_rows: (r,) float32 Q scales; sk_blocks:
-    float32 K scales per 64-key block; scale_log2: float32 sm_scale*log2(e);
+    float32 K scales per kblk-key block; scale_log2: float32 sm_scale*log2(e);
     valid: (r, n_kv) bool key mask; vvals (n_kv, d) and sv (d,) as in
     online_softmax_pv.  The running max m' is the fp32 max of fp32 products of
-    each 64-key half's largest score with that half's scale factor.
+    each K block's largest score with that block's scale factor.
     Returns (out, lse).
     """
     r, n_kv = s_int.shape
     d = vvals.shape[1]
-    nblk = 2 * (-(-n_kv // KV_TILE))
+    per_tile = KV_TILE // kblk
+    nblk = per_tile * (-(-n_kv // KV_TILE))
     skb = np.zeros(nblk, dtype=np.float32)
     skb[:len(sk_blocks)] = sk_blocks
     sq_rows = np.asarray(sq_rows, dtype=np.float32)
@@ -431,11 +435,11 @@ def online_softmax_pv_fp32_decision(s_int, sq_rows, sk_blocks, scale_log2, valid
         cols = np.arange(t0, min(n_kv, t0 + KV_TILE))
         S = s_int[:, cols].astype(np.int64)
         ok = valid[:, cols]
-        half = (cols - t0) // BLKK
-        ck = np.stack([((sq_rows * skb[2 * j + h]).astype(np.float32) * scale_log2).astype(np.float32)
-                       for h in (0, 1)], axis=1)                                   # (r, 2)
+        half = (cols - t0) // kblk                                                 # K block in tile
+        ck = np.stack([((sq_rows * skb[per_tile * j + h]).astype(np.float32) * scale_log2).astype(np.float32)
+                       for h in range(per_tile)], axis=1)                          # (r, per_tile)
         mt = np.full(r, -np.inf, dtype=np.float32)
-        for h in (0, 1):
+        for h in range(per_tile):
             sel = half == h
             if not np.any(sel):
                 continue
@@ -463,7 +467,8 @@ def online_softmax_pv_fp32_decision(s_int, sq_rows, sk_blocks, scale_log2, valid
 
 
 def attention_head_kernel_precision(q, k, v, *, causal=False, sm_scale=None, rows=None,
-                                    quantize_p: bool = True) -> dict:
+                                    quantize_p: bool = True, qblk: int = BLKQ,
+                                    kblk: int = BLKK) -> dict:
     """attention_head with the P8 codes decided in the kernel's fp32 precision.
 
     Quantization of Q, K, V and the integer scores are the same exact stages as
@@ -480,15 +485,15 @@ def attention_head_kernel_precision(q, k, v, *, causal=False, sm_scale=None, row
         raise ValueError("causal attention needs equal query and key lengths")
     rows = np.arange(n) if rows is None else np.asarray(rows, dtype=np.int64)
     mu = k_channel_mean(k)
-    q8, sq = quantize_int8_blocks(q, BLKQ)
-    k8, sk = quantize_int8_blocks(smooth_k(k, mu), BLKK)
+    q8, sq = quantize_int8_blocks(q, qblk)
+    k8, sk = quantize_int8_blocks(smooth_k(k, mu), kblk)
     v8, sv = quantize_v_e4m3(v)
     s_int = integer_scores(q8[rows], k8[:n_kv])
     valid = np.ones((len(rows), n_kv), dtype=bool)
     if causal:
         valid = np.arange(n_kv)[None, :] <= rows[:, None]
     out, lse = online_softmax_pv_fp32_decision(
-        s_int, sq[rows // BLKQ], sk, kernel_scale_log2(d, sm_scale), valid,
-        e4m3_decode(v8), sv.astype(np.float64), quantize_p=quantize_p)
+        s_int, sq[rows // qblk], sk, kernel_scale_log2(d, sm_scale), valid,
+        e4m3_decode(v8), sv.astype(np.float64), quantize_p=quantize_p, kblk=kblk)
     return dict(out=out, lse=lse, rows=rows, k_mean=mu, q8=q8, q_scale=sq, k8=k8, k_scale=sk,
                 v8=v8, v_scale=sv, s_int=s_int)

@@ -108,8 +108,8 @@ def test_k_mean_closed_form():
 
 def test_int8_quantization_is_lossless_on_grid_values():
     rng = np.random.default_rng(2)
-    for blk in (orc.BLKQ, orc.BLKK):
-        n, d = 3 * blk - 17, 64                                  # ragged last block
+    for blk in (orc.BLKQ, orc.BLKK, 32, 1):                    # per block and per thread
+        n, d = 3 * blk - (17 if blk > 17 else 0), 64             # ragged last block
         ints = rng.integers(-126, 127, size=(n, d))
         for b in range(0, n, blk):
             ints[b, 0] = 127 if b % 2 else -127                   # one +-127 per block
@@ -496,3 +496,36 @@ def test_kernel_precision_p8_codes_mostly_equal_fp64_codes():
     diff = p32 != p64
     assert np.all(np.abs(np.log2(p32[diff] / p64[diff])) <= 0.19)
     del u
+
+
+def test_thread_granularity_kernel_precision_path():
+    # per-token Q scales and 32-token K scales (the per-thread granularity): the
+    # kernel-precision path keeps the pins of the per-block one, and on heavy-tailed
+    # input the finer scales are closer to exact attention
+    rng = np.random.default_rng(31)
+    n, d = 300, 64
+    q, k, v = (rng.standard_normal((n, d)).astype(np.float32) for _ in range(3))
+    for t in (q, k):
+        t[rng.random(t.shape) < 0.02] *= 20.0
+    eps = orc.EXP2_MAX_REL_ERR
+    r = orc.attention_head(q, k, v, qblk=1, kblk=32)
+    assert r["q_scale"].shape == (n,) and r["k_scale"].shape == (-(-n // 32),)
+    x = r["s_int"].astype(np.float64) * r["q_scale"][:, None].astype(np.float64) \
+        * r["k_scale"][None, np.arange(n) // 32].astype(np.float64) / math.sqrt(d)
+    vv = orc.e4m3_decode(r["v8"])
+    sv = r["v_scale"].astype(np.float64)
+    ref_unq, _ = orc.online_softmax_pv(x, vv, sv, quantize_p=False)
+    a_unq = orc.attention_head_kernel_precision(q, k, v, quantize_p=False, qblk=1, kblk=32)
+    assert np.max(np.abs(a_unq["out"] - ref_unq)) <= 2.0 * eps / (1.0 - eps) * np.max(np.abs(vv * sv))
+    exact = orc.reference_attention(q, k, v)
+
+    def cos_l1(o):
+        o, e = o.ravel(), exact.ravel()
+        return float(o @ e / (np.linalg.norm(o) * np.linalg.norm(e))), float(np.abs(o - e).sum() / np.abs(e).sum())
+
+    a = orc.attention_head_kernel_precision(q, k, v, qblk=1, kblk=32)
+    cos_a, l1_a = cos_l1(a["out"])
+    cos_b, l1_b = cos_l1(r["out"])
+    assert cos_a >= cos_b - 2e-5 and l1_a <= 1.05 * l1_b
+    cos_blk, l1_blk = cos_l1(orc.attention_head(q, k, v)["out"])
+    assert cos_b > cos_blk and l1_b < l1_blk
