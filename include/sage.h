@@ -40,8 +40,10 @@
  * (dense problems: n_b = seqlen for every b).  Padding entries are written as 0.
  *   q8      int8  [Hq ][T_pad][d]       token t of seq b, head h at (h*T_pad + off_b + t)*d
  *   q_scale float [Hq ][T_pad/128]      one scale per 128-token block of a sequence
+ *                 ([Hq][T_pad], one per token, with SAGE_GRAN_THREAD)
  *   k8      int8  [Hkv][T_pad][d]       smoothed K codes
  *   k_scale float [Hkv][T_pad/64]       one scale per 64-token block of a sequence
+ *                 ([Hkv][T_pad/32], one per 32-token block, with SAGE_GRAN_THREAD)
  *   k_mean  float [B  ][Hkv][d]         per-channel mean of K over the sequence
  *   v8      uint8 [Hkv][d][T_pad]       e4m3 codes, transposed (token-contiguous)
  *   v_scale float [B  ][Hkv][d]         per-channel V scale
@@ -71,6 +73,16 @@ typedef enum {
 
 typedef enum { SAGE_FP16 = 0, SAGE_BF16 = 1, SAGE_FP32 = 2 } sage_dtype_t;
 
+/* Granularity of the INT8 scales of Q and K.
+ * SAGE_GRAN_BLOCK (0, the method as stated): one scale per 128-token Q block and per
+ *   64-token K block of a sequence.
+ * SAGE_GRAN_THREAD (1): finer scales, the reading of the heatdrop review's
+ *   "per-thread quantization" (The interesting bit) for this kernel, where one thread
+ *   owns one query row and takes keys 32 at a time: one scale per Q token and one per
+ *   32-token K block.  Same codes otherwise; the attention kernel folds the scales
+ *   into the same per-row, per-32-key factors. */
+typedef enum { SAGE_GRAN_BLOCK = 0, SAGE_GRAN_THREAD = 1 } sage_granularity_t;
+
 /* Problem description shared by all entry points. */
 typedef struct {
   int batch;              /* B: dense batch size, or number of packed sequences (<= 1024) */
@@ -81,6 +93,7 @@ typedef struct {
   sage_dtype_t dtype;     /* dtype of q, k, v: SAGE_FP16 or SAGE_BF16 */
   const int32_t* cu_seqlens_host; /* host, NULL for dense; else [batch+1] prefix sums of the
                                      packed sequence lengths, cu[0] = 0, non-decreasing */
+  sage_granularity_t granularity; /* INT8 scale granularity of Q and K (zero: per block) */
 } sage_problem_t;
 
 /* Byte sizes of the quantized buffers and of the quantization workspaces. */
@@ -100,7 +113,8 @@ sage_status_t sage_buffer_sizes(const sage_problem_t* p, sage_sizes_t* sizes);
  *  vibecrowd page, How it works: INT8 quantization for QK^T.)
  *   mu[c]  = fp32(sum_t k[t,c] in fp64 / n_b)              per (sequence, kv head)
  *   k_s    = fp32(k - mu)
- *   per block (Q: 128 tokens x d, K: 64 tokens x d of k_s):
+ *   per block (Q: 128 tokens x d, K: 64 tokens x d of k_s; with SAGE_GRAN_THREAD
+ *   Q: 1 token x d, K: 32 tokens x d):
  *     a = max|x|;  s = fp32(a/127);  x8 = clamp(rint_even(fp32(x * fp32(127/a))), -127, 127)
  *     (a == 0: s = 0, codes 0)
  * Writes q8, q_scale, k8, k_scale, k_mean (layouts above).  `workspace` must
@@ -155,7 +169,8 @@ sage_status_t sage_quant_v(const sage_problem_t* p, const void* v, const int64_t
  * (vibecrowd page, How it works; heatdrop review, The interesting bit and Key highlights.)
  * For each query row i of sequence b, head h (KV head h/(Hq/Hkv)), over KV blocks of
  * 128 keys in order:
- *   x_j  = S_ij * q_scale * k_scale_j * sm_scale   (S_ij exact int32 from INT8 MMAs)
+ *   x_j  = S_ij * q_scale_i * k_scale_j * sm_scale (S_ij exact int32 from INT8 MMAs; the
+ *          scales of row i's Q block and key j's K block at the problem's granularity)
  *   causal: x_j = -inf for j > i
  *   m'   = max(m, max_j x_j);   P~_j = exp(x_j - m');   l = l e^{m-m'} + sum_j P~_j
  *   P8   = e4m3(448 P~);  PV_blk = P8 V8 (FP32, fresh per block);  O = O e^{m-m'} + PV_blk

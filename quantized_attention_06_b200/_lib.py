@@ -19,6 +19,7 @@ SAGE_ERR_TOO_LARGE = 5
 NOALLOC_SCRATCH_BYTES = 8 << 20  # SAGE_NOALLOC_SCRATCH_BYTES
 
 SAGE_FP16, SAGE_BF16, SAGE_FP32 = 0, 1, 2
+SAGE_GRAN_BLOCK, SAGE_GRAN_THREAD = 0, 1
 
 EXPORTS = (
     "sage_buffer_sizes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd",
@@ -36,6 +37,7 @@ class SageProblem(ctypes.Structure):
         ("head_dim", ctypes.c_int),
         ("dtype", ctypes.c_int),
         ("cu_seqlens_host", ctypes.POINTER(ctypes.c_int32)),
+        ("granularity", ctypes.c_int),  # SAGE_GRAN_BLOCK / SAGE_GRAN_THREAD
     ]
 
 

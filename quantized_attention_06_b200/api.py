@@ -26,6 +26,9 @@ __all__ = ["Problem", "Quantized", "quant_qk", "quant_qk_noalloc", "quant_v", "a
            "sageattn", "sageattn_host", "debug_qk_int32", "poll_device_status"]
 
 _IN_DTYPES = {torch.float16: L.SAGE_FP16, torch.bfloat16: L.SAGE_BF16}
+# INT8 scale granularity of Q and K: "block" (128-token Q / 64-token K blocks, the
+# method as stated) or "thread" (a scale per Q token and per 32-token K block)
+_GRANULARITY = {"block": L.SAGE_GRAN_BLOCK, "thread": L.SAGE_GRAN_THREAD}
 _OUT_DTYPES = {torch.float16: L.SAGE_FP16, torch.bfloat16: L.SAGE_BF16, torch.float32: L.SAGE_FP32}
 
 
@@ -40,9 +43,13 @@ def _stream() -> ctypes.c_void_p:
 class Problem:
     """Shapes of one attention call (sage_problem_t)."""
 
-    def __init__(self, batch, heads_q, heads_kv, seqlen, head_dim, dtype, cu_seqlens=None):
+    def __init__(self, batch, heads_q, heads_kv, seqlen, head_dim, dtype, cu_seqlens=None,
+                 granularity="block"):
         if dtype not in _IN_DTYPES:
             raise TypeError(f"q/k/v must be float16 or bfloat16, got {dtype}")
+        if granularity not in _GRANULARITY:
+            raise ValueError(f"granularity must be 'block' or 'thread', got {granularity!r}")
+        self.granularity = granularity
         self.dtype = dtype
         self.varlen = cu_seqlens is not None
         if self.varlen:
@@ -55,7 +62,8 @@ class Problem:
         else:
             self.cu_list = None
             cu_ptr = ctypes.POINTER(ctypes.c_int32)()
-        self.c = L.SageProblem(batch, heads_q, heads_kv, seqlen, head_dim, _IN_DTYPES[dtype], cu_ptr)
+        self.c = L.SageProblem(batch, heads_q, heads_kv, seqlen, head_dim, _IN_DTYPES[dtype], cu_ptr,
+                               _GRANULARITY[granularity])
         self.batch, self.heads_q, self.heads_kv = batch, heads_q, heads_kv
         self.seqlen, self.head_dim = seqlen, head_dim
         sz = L.SageSizes()
@@ -63,12 +71,20 @@ class Problem:
         self.sizes = sz
         self.t_pad = int(sz.t_pad)
 
+    @property
+    def q_block(self) -> int:
+        return 1 if self.granularity == "thread" else 128
+
+    @property
+    def k_block(self) -> int:
+        return 32 if self.granularity == "thread" else 64
+
     @staticmethod
-    def from_tensors(q, k, tensor_layout="HND", cu_seqlens=None) -> "Problem":
+    def from_tensors(q, k, tensor_layout="HND", cu_seqlens=None, granularity="block") -> "Problem":
         if cu_seqlens is not None:
             _, hq, d = q.shape
             hkv = k.shape[1]
-            return Problem(0, hq, hkv, 0, d, q.dtype, cu_seqlens)
+            return Problem(0, hq, hkv, 0, d, q.dtype, cu_seqlens, granularity)
         if tensor_layout == "HND":
             b, hq, n, d = q.shape
             hkv = k.shape[1]
@@ -77,7 +93,7 @@ class Problem:
             hkv = k.shape[2]
         else:
             raise ValueError(f"tensor_layout must be 'HND' or 'NHD', got {tensor_layout!r}")
-        return Problem(b, hq, hkv, n, d, q.dtype)
+        return Problem(b, hq, hkv, n, d, q.dtype, granularity=granularity)
 
 
 def _strides(t: torch.Tensor, tensor_layout: str, varlen: bool):
@@ -117,19 +133,19 @@ def _require_cuda(*ts):
 
 
 def quant_qk(q, k, tensor_layout="HND", cu_seqlens=None, problem=None, out: Quantized = None,
-             workspace=None) -> Quantized:
+             workspace=None, granularity="block") -> Quantized:
     """K smoothing + per-block INT8 quantization of Q and K (sage_quant_qk)."""
     _require_cuda(q, k)
-    p = problem or Problem.from_tensors(q, k, tensor_layout, cu_seqlens)
+    p = problem or Problem.from_tensors(q, k, tensor_layout, cu_seqlens, granularity)
     z = out or Quantized(p, tensor_layout)
     dev = q.device
     sz = p.sizes
     d, tp = p.head_dim, p.t_pad
     if z.q8 is None:
         z.q8 = torch.empty((p.heads_q, tp, d), dtype=torch.int8, device=dev)
-        z.q_scale = torch.empty((p.heads_q, tp // 128), dtype=torch.float32, device=dev)
+        z.q_scale = torch.empty((p.heads_q, tp // p.q_block), dtype=torch.float32, device=dev)
         z.k8 = torch.empty((p.heads_kv, tp, d), dtype=torch.int8, device=dev)
-        z.k_scale = torch.empty((p.heads_kv, tp // 64), dtype=torch.float32, device=dev)
+        z.k_scale = torch.empty((p.heads_kv, tp // p.k_block), dtype=torch.float32, device=dev)
         z.k_mean = torch.empty((p.batch, p.heads_kv, d), dtype=torch.float32, device=dev)
     ws = workspace if workspace is not None else _alloc(sz.workspace_qk, torch.float64, dev)
     varlen = p.varlen
@@ -143,21 +159,21 @@ def quant_qk(q, k, tensor_layout="HND", cu_seqlens=None, problem=None, out: Quan
 
 
 def quant_qk_noalloc(q, k, tensor_layout="HND", cu_seqlens=None, problem=None,
-                     out: Quantized = None) -> Quantized:
+                     out: Quantized = None, granularity="block") -> Quantized:
     """quant_qk without a workspace (sage_quant_qk_noalloc), for callers that cannot
     allocate device memory when they quantize.  The scratch comes from a fixed
     library-owned device array; ``out`` should then hold preallocated outputs.
     Calls that overlap on the GPU race on that shared scratch."""
     _require_cuda(q, k)
-    p = problem or Problem.from_tensors(q, k, tensor_layout, cu_seqlens)
+    p = problem or Problem.from_tensors(q, k, tensor_layout, cu_seqlens, granularity)
     z = out or Quantized(p, tensor_layout)
     dev = q.device
     d, tp = p.head_dim, p.t_pad
     if z.q8 is None:
         z.q8 = torch.empty((p.heads_q, tp, d), dtype=torch.int8, device=dev)
-        z.q_scale = torch.empty((p.heads_q, tp // 128), dtype=torch.float32, device=dev)
+        z.q_scale = torch.empty((p.heads_q, tp // p.q_block), dtype=torch.float32, device=dev)
         z.k8 = torch.empty((p.heads_kv, tp, d), dtype=torch.int8, device=dev)
-        z.k_scale = torch.empty((p.heads_kv, tp // 64), dtype=torch.float32, device=dev)
+        z.k_scale = torch.empty((p.heads_kv, tp // p.k_block), dtype=torch.float32, device=dev)
         z.k_mean = torch.empty((p.batch, p.heads_kv, d), dtype=torch.float32, device=dev)
     st = L.lib().sage_quant_qk_noalloc(
         ctypes.byref(p.c), _ptr(q), _strides(q, tensor_layout, p.varlen),
@@ -212,9 +228,10 @@ def attn_fwd(z: Quantized, is_causal=False, sm_scale=None, out_dtype=None, out=N
 
 
 def sageattn(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, cu_seqlens=None,
-             out_dtype=None, return_lse=False):
-    """Quantized attention: smoothing + INT8 Q/K, FP8 V, then the fused attention kernel."""
-    z = quant_qk(q, k, tensor_layout, cu_seqlens)
+             out_dtype=None, return_lse=False, granularity="block"):
+    """Quantized attention: smoothing + INT8 Q/K, FP8 V, then the fused attention kernel.
+    granularity="thread" selects a Q scale per token and a K scale per 32 tokens."""
+    z = quant_qk(q, k, tensor_layout, cu_seqlens, granularity=granularity)
     quant_v(v, z)
     return attn_fwd(z, is_causal=is_causal, sm_scale=sm_scale, out_dtype=out_dtype,
                     return_lse=return_lse)
@@ -224,7 +241,8 @@ _HOST_WS = {}
 
 
 def sageattn_host(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, out=None,
-                  out_dtype=None, kv_heads_per_chunk=0, device=None, synchronize=True):
+                  out_dtype=None, kv_heads_per_chunk=0, device=None, synchronize=True,
+                  granularity="block"):
     """sageattn on host tensors (sage_attn_host): chunks of heads are copied in,
     computed and copied out with the copies overlapping the kernels.
 
@@ -250,7 +268,7 @@ def sageattn_host(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, 
         code = 1
     else:
         raise ValueError(f"tensor_layout must be HND or NHD, got {tensor_layout}")
-    p = Problem(b, hq, hkv, n, d, q.dtype)
+    p = Problem(b, hq, hkv, n, d, q.dtype, granularity=granularity)
     odt = out_dtype or q.dtype
     if odt not in _OUT_DTYPES:
         raise TypeError(f"unsupported output dtype {odt}")

@@ -73,6 +73,7 @@ struct AttnArgs {
   int hq, hkv, group;
   float scale_log2;  // sm_scale * log2(e)
   int causal;
+  int fine;  // per-thread granularity: q_scale per token, k_scale per 32-token block
 };
 
 template <int D>
@@ -181,7 +182,7 @@ __device__ __forceinline__ f2 pair_of(const uint32_t (&r)[32], int k) {
 constexpr uint32_t kMagicBits = 0x4B400000u;
 constexpr float kMagic = 12582912.0f;
 
-// max over 32 magic-offset scores (masked entries hold 0, below every valid value)
+// max of acc and 32 magic-offset scores (masked entries hold 0, below every valid value)
 __device__ __forceinline__ float max32(const uint32_t (&r)[32], float acc) {
   float m0 = acc, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
 #pragma unroll
@@ -448,8 +449,14 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t c0 = 64u * h;    // this half's S columns; its P8 takes the first 16
     bool ok = !dead;
-    const float sq = a.q_scale[static_cast<int64_t>(hq) * (seq.t_pad / kBlkQ) + off / kBlkQ + qt];
-    const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kBlkK) + off / kBlkK;
+    // this row's Q scale, and the K scales of the sequence; ksc32(j, c) is the scale of
+    // keys 32c .. 32c + 31 of KV tile j (its 64-token block, or its own 32-token block)
+    const float sq = a.fine
+        ? a.q_scale[static_cast<int64_t>(hq) * seq.t_pad + off + qt * kBlkQ + row]
+        : a.q_scale[static_cast<int64_t>(hq) * (seq.t_pad / kBlkQ) + off / kBlkQ + qt];
+    const int kblk = a.fine ? kBlkKFine : kBlkK;
+    const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kblk) + off / kblk;
+    auto ksc32 = [&](int j, int c) { return a.fine ? ksc[4 * j + c] : ksc[2 * j + (c >> 1)]; };
 
     // both S buffers start free
     if (ok && lane == 0) { mbar_arrive(bar_sfree(0)); mbar_arrive(bar_sfree(1)); }
@@ -458,9 +465,9 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     for (int j = 0; j < nkv && ok; ++j) {
       const int buf = j & 1;
       const uint32_t tS = tmem + lane_base + 128u * buf;
-      const float ck0 = __fmul_rn(__fmul_rn(sq, ksc[2 * j]), a.scale_log2);
-      const float ck1 = __fmul_rn(__fmul_rn(sq, ksc[2 * j + 1]), a.scale_log2);
-      const float ck = h ? ck1 : ck0;
+      // logit factors of this half's two 32-key chunks
+      const float cka = __fmul_rn(__fmul_rn(sq, ksc32(j, 2 * h)), a.scale_log2);
+      const float ckb = __fmul_rn(__fmul_rn(sq, ksc32(j, 2 * h + 1)), a.scale_log2);
       const bool masked = (a.causal && j == qt) || (j + 1) * kKvTile > n;
       const int kv0 = j * kKvTile + 64 * h;  // first key of this half
       auto dropped = [&](int key) { return key >= n || (a.causal && key > grow); };
@@ -484,17 +491,19 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
           if (dropped(kv0 + 32 + i)) rb[i] = 0u; else keep_b |= 1u << i;
         }
       }
-      const float hm = max32(rb, max32(ra, 0.0f));
-      // exchange half maxima with the other softmax warp of this lane quarter
-      xchg[(buf * 2 + h) * 128 + row] = hm;
+      // this half's max logit (log2 units): each 32-key chunk's largest score times the
+      // chunk's factor (the same as the largest score of the half times its factor when
+      // both chunks share one K block: rounding is monotone)
+      const float hma = max32(ra, 0.0f), hmb = max32(rb, 0.0f);
+      const float hs = fmaxf(hma > 1.0e6f ? __fmul_rn(__fsub_rn(hma, kMagic), cka) : -INFINITY,
+                             hmb > 1.0e6f ? __fmul_rn(__fsub_rn(hmb, kMagic), ckb) : -INFINITY);
+      // exchange with the other softmax warp of this lane quarter
+      xchg[(buf * 2 + h) * 128 + row] = hs;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_xchg(buf, quarter));
       ok = __all_sync(0xffffffffu, mbar_wait(bar_xchg(buf, quarter), (j >> 1) & 1, 0x305 + h));
       if (!ok) break;
-      const float ho = xchg[(buf * 2 + (1 - h)) * 128 + row];
-      const float hmax0 = h ? ho : hm, hmax1 = h ? hm : ho;
-      const float mt = fmaxf(hmax0 > 1.0e6f ? __fmul_rn(__fsub_rn(hmax0, kMagic), ck0) : -INFINITY,
-                             hmax1 > 1.0e6f ? __fmul_rn(__fsub_rn(hmax1, kMagic), ck1) : -INFINITY);
+      const float mt = fmaxf(hs, xchg[(buf * 2 + (1 - h)) * 128 + row]);
       const float m_new = fmaxf(m, mt);
       const float alpha = ex2(m - m_new);
       const float nbias = __fsub_rn(kLog2_448, m_new);
@@ -504,11 +513,11 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       // first 16 columns
       f2 acc = make_float2(0.0f, 0.0f);
       uint32_t w[8];
-      if (masked) p8_chunk<true>(ra, ck, nbias, acc, w, keep_a);
-      else p8_chunk<false>(ra, ck, nbias, acc, w, 0u);
+      if (masked) p8_chunk<true>(ra, cka, nbias, acc, w, keep_a);
+      else p8_chunk<false>(ra, cka, nbias, acc, w, 0u);
       tmem_st8(tS + c0, w);
-      if (masked) p8_chunk<true>(rb, ck, nbias, acc, w, keep_b);
-      else p8_chunk<false>(rb, ck, nbias, acc, w, 0u);
+      if (masked) p8_chunk<true>(rb, ckb, nbias, acc, w, keep_b);
+      else p8_chunk<false>(rb, ckb, nbias, acc, w, 0u);
       tmem_st8(tS + c0 + 8u, w);
       l = l * alpha + (f2_lo(acc) + f2_hi(acc));
       m = m_new;

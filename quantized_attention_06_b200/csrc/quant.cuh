@@ -156,6 +156,7 @@ struct QKQuantArgs {
   const float* k_mean;
   int hq, hkv;
   int nq_blocks;  // hq * t_pad / 128 (the first CTAs); the rest are K blocks
+  int fine;       // per-thread granularity: a scale per Q token and per 32-token K block
 };
 
 __device__ __forceinline__ float block_max_256(float v, float* red) {
@@ -186,6 +187,7 @@ quant_qk_kernel(const __grid_constant__ Seq seq, const __grid_constant__ QKQuant
   constexpr int VPR = D / 8;
   constexpr int RG = kQuantThreads / VPR;
   constexpr int ITQ = kBlkQ / RG;  // 8 (d=128) or 4 (d=64)
+  static_assert(RG == 16 || RG == 32, "a row group must not straddle a 32-row K block");
   __shared__ float red[kQuantThreads / 32];
   const bool isq = static_cast<int>(blockIdx.x) < a.nq_blocks;
   const int rows = isq ? kBlkQ : kBlkK;
@@ -223,14 +225,68 @@ quant_qk_kernel(const __grid_constant__ Seq seq, const __grid_constant__ QKQuant
       amax = fmaxf(amax, fabsf(x[it][i]));
     }
   }
-  amax = block_max_256(amax, red);
-  const float s = (amax > 0.0f) ? __fdiv_rn(amax, 127.0f) : 0.0f;
-  const float r = (amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
+  // the scale of each row: one per CTA block, or (fine) one per Q row / 32-row K block
+  float rit[ITQ];
   int8_t* dst = (isq ? a.q8 : a.k8) + (static_cast<int64_t>(h) * seq.t_pad + tp) * D + vc * 8;
+  if (!a.fine) {
+    amax = block_max_256(amax, red);
+    const float s = (amax > 0.0f) ? __fdiv_rn(amax, 127.0f) : 0.0f;
+    const float r = (amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
+#pragma unroll
+    for (int it = 0; it < ITQ; ++it) rit[it] = r;
+    if (threadIdx.x == 0) (isq ? a.q_scale : a.k_scale)[static_cast<int64_t>(h) * per_head + pb] = s;
+  } else if (isq) {
+    // the VPR consecutive lanes holding one row reduce its max by shuffles
+#pragma unroll
+    for (int it = 0; it < ITQ; ++it) {
+      float m = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[it][i]));
+#pragma unroll
+      for (int o = VPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      rit[it] = (m > 0.0f) ? __fdiv_rn(127.0f, m) : 0.0f;
+      if (vc == 0 && it < iters)
+        a.q_scale[static_cast<int64_t>(h) * seq.t_pad + tp + rg + it * RG] =
+            (m > 0.0f) ? __fdiv_rn(m, 127.0f) : 0.0f;
+    }
+  } else {
+    // two 32-row K blocks per CTA: row rg + it * RG (rg < RG) lies in block it * RG / 32
+    __shared__ float red2[2][kQuantThreads / 32];
+    float m2[2] = {0.0f, 0.0f};
+#pragma unroll
+    for (int it = 0; it < ITQ; ++it) {
+      if (it < iters) {
+        const int sb = (it * RG) / kBlkKFine;  // rows it*RG .. it*RG + RG-1, RG in {16, 32}
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m2[sb] = fmaxf(m2[sb], fabsf(x[it][i]));
+      }
+    }
+#pragma unroll
+    for (int b2 = 0; b2 < 2; ++b2) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m2[b2] = fmaxf(m2[b2], __shfl_xor_sync(0xffffffffu, m2[b2], o));
+      if ((threadIdx.x & 31) == 0) red2[b2][threadIdx.x >> 5] = m2[b2];
+    }
+    __syncthreads();
+    float r2[2];
+#pragma unroll
+    for (int b2 = 0; b2 < 2; ++b2) {
+      float m = red2[b2][0];
+#pragma unroll
+      for (int i = 1; i < kQuantThreads / 32; ++i) m = fmaxf(m, red2[b2][i]);
+      r2[b2] = (m > 0.0f) ? __fdiv_rn(127.0f, m) : 0.0f;
+      if (threadIdx.x == 0)
+        a.k_scale[static_cast<int64_t>(h) * (seq.t_pad / kBlkKFine) + pb * 2 + b2] =
+            (m > 0.0f) ? __fdiv_rn(m, 127.0f) : 0.0f;
+    }
+#pragma unroll
+    for (int it = 0; it < ITQ; ++it) rit[it] = r2[((it * RG) / kBlkKFine) & 1];
+  }
 #pragma unroll
   for (int it = 0; it < ITQ; ++it) {
     if (it < iters) {
       const int rr = rg + it * RG;
+      const float r = rit[it];
       uint2 o;
       o.x = pack_i8x4(quant_i8(x[it][0], r), quant_i8(x[it][1], r), quant_i8(x[it][2], r),
                       quant_i8(x[it][3], r));
@@ -239,7 +295,6 @@ quant_qk_kernel(const __grid_constant__ Seq seq, const __grid_constant__ QKQuant
       *reinterpret_cast<uint2*>(dst + static_cast<int64_t>(rr) * D) = o;
     }
   }
-  if (threadIdx.x == 0) (isq ? a.q_scale : a.k_scale)[static_cast<int64_t>(h) * per_head + pb] = s;
 }
 
 // ------------------------------------------------------------------------- V e4m3

@@ -17,6 +17,7 @@ namespace sage {
 // Quantization / tiling constants shared by every kernel of the library.
 constexpr int kBlkQ = 128;    // tokens per Q quantization block = query rows per tile
 constexpr int kBlkK = 64;     // tokens per K quantization block
+constexpr int kBlkKFine = 32; // tokens per K block with per-thread granularity
 constexpr int kKvTile = 128;  // keys per online-softmax block (KV tile)
 constexpr int kPad = 128;     // every sequence is padded to a multiple of this
 

@@ -40,6 +40,8 @@ sage_status_t plan(const sage_problem_t* p, Layout& L, SeqVarlen* storage) {
   if (p->heads_q % p->heads_kv != 0) return SAGE_ERR_INVALID_ARGUMENT;
   if (p->head_dim != 64 && p->head_dim != 128) return SAGE_ERR_UNSUPPORTED;
   if (p->dtype != SAGE_FP16 && p->dtype != SAGE_BF16) return SAGE_ERR_UNSUPPORTED;
+  if (p->granularity != SAGE_GRAN_BLOCK && p->granularity != SAGE_GRAN_THREAD)
+    return SAGE_ERR_INVALID_ARGUMENT;
   L.nseq = p->batch;
   if (p->cu_seqlens_host == nullptr) {
     if (p->seqlen < 1) return SAGE_ERR_INVALID_ARGUMENT;
@@ -159,6 +161,7 @@ sage_status_t launch_quant_qk(const Seq& seq, const sage_problem_t* p, int64_t t
   a.q8 = q8; a.q_scale = q_scale; a.k8 = k8; a.k_scale = k_scale; a.k_mean = k_mean;
   a.hq = p->heads_q; a.hkv = p->heads_kv;
   a.nq_blocks = static_cast<int>(p->heads_q * (t_pad / kBlkQ));
+  a.fine = p->granularity == SAGE_GRAN_THREAD ? 1 : 0;
   const int nk_blocks = static_cast<int>(p->heads_kv * (t_pad / kBlkK));
   quant_qk_kernel<T, D, Seq><<<a.nq_blocks + nk_blocks, kQuantThreads, 0, st>>>(seq, a);
   return launched();
@@ -223,9 +226,10 @@ sage_status_t sage_buffer_sizes(const sage_problem_t* p, sage_sizes_t* sz) {
   const size_t d = p->head_dim, tp = static_cast<size_t>(L.t_pad);
   sz->t_pad = tp;
   sz->q8 = static_cast<size_t>(p->heads_q) * tp * d;
-  sz->q_scale = static_cast<size_t>(p->heads_q) * (tp / kBlkQ) * sizeof(float);
+  const bool fine = p->granularity == SAGE_GRAN_THREAD;
+  sz->q_scale = static_cast<size_t>(p->heads_q) * (tp / (fine ? 1 : kBlkQ)) * sizeof(float);
   sz->k8 = static_cast<size_t>(p->heads_kv) * tp * d;
-  sz->k_scale = static_cast<size_t>(p->heads_kv) * (tp / kBlkK) * sizeof(float);
+  sz->k_scale = static_cast<size_t>(p->heads_kv) * (tp / (fine ? kBlkKFine : kBlkK)) * sizeof(float);
   sz->k_mean = static_cast<size_t>(p->batch) * p->heads_kv * d * sizeof(float);
   sz->v8 = static_cast<size_t>(p->heads_kv) * d * tp;
   sz->v_scale = sz->k_mean;
@@ -326,6 +330,7 @@ sage_status_t sage_attn_fwd(const sage_problem_t* p, const int8_t* q8, const flo
   const float scale = sm_scale > 0.0f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(d));
   a.scale_log2 = scale * kLog2E;
   a.causal = is_causal ? 1 : 0;
+  a.fine = p->granularity == SAGE_GRAN_THREAD ? 1 : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (L.varlen) {
     const int64_t ncta = L.var->cta[p->batch];
