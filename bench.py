@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--causal", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=1536)
+    ap.add_argument("--granularity", default="block", choices=["block", "thread"],
+                    help="INT8 scale granularity of Q/K: per block (the method as stated) or "
+                         "per thread (a scale per Q token and per 32-token K block)")
     return ap.parse_args()
 
 
@@ -59,7 +62,8 @@ def config(w, args, n_gpus):
             "batch": w.batch, "heads": w.heads_q, "seq_len": w.seqlen, "head_dim": w.head_dim,
             "causal": bool(args.causal), "layout": w.layout, "n_gpus": n_gpus,
             "l2": "inputs (3 x 256 MiB) larger than the 126 MB L2; no flush",
-            "step": "sage_quant_qk + sage_quant_v + sage_attn_fwd"}
+            "step": "sage_quant_qk + sage_quant_v + sage_attn_fwd",
+            "granularity": getattr(args, "granularity", "block")}
 
 
 def peaks():
@@ -80,7 +84,9 @@ def cpu_sample(w, args, rows):
     q, k, v = x["q"][0, 0], x["k"][0, 0], x["v"][0, 0]
     sel = np.linspace(0, w.seqlen - 1, rows).astype(np.int64)
     t0 = time.perf_counter()
-    orc.attention_head_kernel_precision(q, k, v, causal=args.causal, rows=sel)
+    thread = getattr(args, "granularity", "block") == "thread"
+    orc.attention_head_kernel_precision(q, k, v, causal=args.causal, rows=sel,
+                                        qblk=1 if thread else orc.BLKQ, kblk=32 if thread else orc.BLKK)
     dt = time.perf_counter() - t0
     n_keys = (sel + 1).sum() if args.causal else rows * w.seqlen
     ops = 4.0 * n_keys * w.head_dim
@@ -198,7 +204,7 @@ def run_sage(args):
     host = {n: torch.from_numpy(x[n]).to(torch.float16).pin_memory() for n in ("q", "k", "v")}
     del x
     q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
-    p = api.Problem.from_tensors(q, k, "HND")
+    p = api.Problem.from_tensors(q, k, "HND", granularity=args.granularity)
     z = api.Quantized(p, "HND")
     ws_qk = torch.empty(max(1, p.sizes.workspace_qk // 8), dtype=torch.float64, device=dev)
     ws_v = torch.empty(max(1, p.sizes.workspace_v // 4), dtype=torch.float32, device=dev)
@@ -260,7 +266,8 @@ def run_sage(args):
             # the public host-buffer call: chunks of heads are copied in, quantized,
             # attended and copied out, with the copies overlapping the kernels
             api.sageattn_host(host["q"], host["k"], host["v"], tensor_layout="HND",
-                              is_causal=args.causal, out=host_out, synchronize=False)
+                              is_causal=args.causal, out=host_out, synchronize=False,
+                              granularity=args.granularity)
 
         e2e_step()
         barrier()
