@@ -104,6 +104,25 @@ def threads_used():
         return 1
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of each rank's `values` over all ranks (the slowest rank sets
+    the job's time); every rank calls it at the same point.  Without a process group
+    (one rank) the values come back unchanged."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(x) for x in values]
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_rate(ops_per_rank, world, ms):
+    """Whole-job TOPS: every rank runs the same workload (weak scaling), so the job
+    does ops_per_rank * world in the slowest rank's `ms` milliseconds."""
+    return ops_per_rank * world / (ms * 1e-3) / 1e12
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -244,17 +263,12 @@ def run_sage(args):
         barrier()
     total_ms = t_start.elapsed_time(t_end)
     attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
-    if world > 1:
-        tt = torch.tensor([total_ms, statistics.mean(attn_ms)], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms, attn_mean = tt.tolist()
-    else:
-        attn_mean = statistics.mean(attn_ms)
+    total_ms, attn_mean = max_over_ranks([total_ms, statistics.mean(attn_ms)], dev)
     assert api.poll_device_status() == 0
 
     ops = w.ops(args.causal)
     ms_per_step = total_ms / args.steps
-    value = ops * world / (ms_per_step * 1e-3) / 1e12
+    value = job_rate(ops, world, ms_per_step)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -277,13 +291,9 @@ def run_sage(args):
             e2e_step()
         e1.record(stream)
         barrier()
-        e_ms = e0.elapsed_time(e1) / e_steps
-        if world > 1:
-            tt = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = tt.item()
+        e_ms, = max_over_ranks([e0.elapsed_time(e1) / e_steps], dev)
         h2d = sum(t.numel() * t.element_size() for t in host.values())
-        e2e = {"value": ops * world / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_rate(ops, world, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out.numel() * out.element_size(),
                "ms_per_step": e_ms}
 
