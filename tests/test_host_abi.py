@@ -156,3 +156,27 @@ def test_host_pipeline_workspace_and_validation(lib):
 def test_host_pipeline_without_gpu_fails_loudly(lib):
     p = _problem(b=1, hq=2, hkv=2, n=256, d=64)
     assert _attn_host(lib, p) == L.SAGE_ERR_CUDA
+
+
+def test_granularity_sizes_and_validation(lib):
+    p = _problem(b=2, hq=4, hkv=2, n=300, d=128)
+    p.granularity = L.SAGE_GRAN_THREAD
+    st, s = _sizes(lib, p)
+    assert st == 0
+    tp = 2 * 384
+    assert s.q_scale == 4 * tp * 4 and s.k_scale == 2 * (tp // 32) * 4   # per token / per 32
+    assert s.q8 == 4 * tp * 128 and s.k8 == 2 * tp * 128                   # codes unchanged
+    for bad in (2, -1, 7):
+        p.granularity = bad
+        assert _sizes(lib, p)[0] == L.SAGE_ERR_INVALID_ARGUMENT
+        assert _quant_qk(lib, p) == L.SAGE_ERR_INVALID_ARGUMENT
+
+
+def test_python_problem_granularity():
+    from quantized_attention_06_b200 import api
+    p = api.Problem(1, 2, 2, 300, 64, torch.float16, granularity="thread")
+    assert p.q_block == 1 and p.k_block == 32 and p.c.granularity == L.SAGE_GRAN_THREAD
+    assert p.sizes.q_scale == 2 * p.t_pad * 4
+    assert api.Problem(1, 2, 2, 300, 64, torch.float16).k_block == 64
+    with pytest.raises(ValueError):
+        api.Problem(1, 2, 2, 300, 64, torch.float16, granularity="warp")
