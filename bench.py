@@ -152,7 +152,10 @@ class Clocks:
     def __init__(self, dev_index):
         self.dev = dev_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        # the per-sample log; SAGE_CLOCKS_DIR keeps it somewhere chosen, else a temp dir
+        import tempfile
+        base = os.environ.get("SAGE_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(base, f"clocks_bench_{os.getpid()}.csv")
 
     def __enter__(self):
         os.makedirs(os.path.dirname(self.path), exist_ok=True)

@@ -23,10 +23,11 @@ Everything after the integer scores is done in float64, with one exception
 kept apart in ``attention_head_kernel_precision``: P8 is an integer code decided
 by floating point, so for GPU parity that decision is taken with the kernel's
 own fp32 steps (fp32 logits and running max, t = fma(S, ck, log2 448 - m'),
-the documented fp32 exp2 algorithm, e4m3 rounding); l, the rescale factors, PV
-and the output stay fp64.  ``attention_head`` is the all-fp64 definition.
+the documented fp32 exp2 algorithm, e4m3 rounding); the row sum l adds the same
+unrounded p, and the sums, rescale factors, PV and the output stay fp64.
+``attention_head`` is the all-fp64 definition.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * Q blocks are 128 tokens x d, K blocks are 64 tokens x d, per (sequence, head);
   the last block of a sequence may be short (its max ignores absent tokens).
@@ -41,6 +42,9 @@ Readings where the pages are silent (each is listed in the design doc):
 * GQA: query head h reads KV head h // (Hq / Hkv).  Varlen: every packed
   sequence is an independent problem (its own mean, blocks and causal diagonal).
 * Causal (equal query and key lengths): key j is masked for query i when j > i.
+* "Per-thread quantization" (heatdrop review, The interesting bit) is read as a Q
+  scale per token and a K scale per 32-token block (qblk = 1, kblk = 32), an option
+  next to the per-block default.
 
 Parity of every function here is pinned by ``tests/test_oracle_pins.py``:
 brute force on tiny inputs, closed forms, invariants and the OCP FP8 value table.
