@@ -529,3 +529,25 @@ def test_thread_granularity_kernel_precision_path():
     assert cos_a >= cos_b - 2e-5 and l1_a <= 1.05 * l1_b
     cos_blk, l1_blk = cos_l1(orc.attention_head(q, k, v)["out"])
     assert cos_b > cos_blk and l1_b < l1_blk
+
+
+def test_running_max_per_32_key_block_equals_per_half_when_scales_agree():
+    # The kernel takes the row max per 32-key chunk (largest score times the chunk's
+    # factor) in both granularities.  With the per-block default both chunks of a
+    # 64-key half share one factor, and fp32 rounding is monotone, so the result must
+    # equal the per-half max exactly: here kblk = 32 with each pair of 32-block scales
+    # equal reproduces kblk = 64 bit for bit.
+    rng = np.random.default_rng(41)
+    r, n_kv, d = 50, 300, 16
+    s_int = rng.integers(-2_000_000, 2_000_000, size=(r, n_kv)).astype(np.int32)
+    sq = rng.uniform(0.01, 0.05, size=r).astype(np.float32)
+    sk64 = rng.uniform(0.01, 0.05, size=-(-n_kv // 64)).astype(np.float32)
+    sk32 = np.repeat(sk64, 2)[:-(-n_kv // 32)]
+    valid = rng.random((r, n_kv)) < 0.9
+    valid[:, 0] = True
+    vv = rng.standard_normal((n_kv, d))
+    sv = np.ones(d)
+    sc = orc.kernel_scale_log2(64)
+    a = orc.online_softmax_pv_fp32_decision(s_int, sq, sk64, sc, valid, vv, sv, kblk=64)
+    b = orc.online_softmax_pv_fp32_decision(s_int, sq, sk32, sc, valid, vv, sv, kblk=32)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
