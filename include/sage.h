@@ -233,6 +233,17 @@ sage_status_t sage_attn_host(const sage_problem_t* p, int tensor_layout,
                              size_t workspace_bytes, sage_stream_t stream);
 
 /*
+ * sage_debug_watchdog_selftest - test hook for the failure path of the bounded waits.
+ * Launches one 32-thread CTA whose first thread waits on an mbarrier phase that
+ * nothing completes, checking the clock as the kernels' waits do, and gives up after
+ * limit_us microseconds (1 .. 1000000): it records SAGE_ERR_DEVICE_TIMEOUT in the
+ * device watchdog word and returns.  No fault and no hang: the next
+ * sage_poll_device_status() reports the timeout and clears the word, and the
+ * context stays usable.  SAGE_ERR_INVALID_ARGUMENT for a limit out of range.
+ */
+sage_status_t sage_debug_watchdog_selftest(unsigned int limit_us, sage_stream_t stream);
+
+/*
  * Synchronize `stream`, then read and clear the device watchdog word of the
  * current device.  Returns SAGE_OK, SAGE_ERR_DEVICE_TIMEOUT or SAGE_ERR_CUDA.
  */

@@ -24,7 +24,8 @@ SAGE_GRAN_BLOCK, SAGE_GRAN_THREAD = 0, 1
 EXPORTS = (
     "sage_buffer_sizes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd",
     "sage_debug_qk_int32", "sage_poll_device_status", "sage_quant_qk_noalloc",
-    "sage_attn_host", "sage_host_workspace_bytes", "sage_status_string",
+    "sage_attn_host", "sage_host_workspace_bytes", "sage_debug_watchdog_selftest",
+    "sage_status_string",
 )
 
 
@@ -76,6 +77,7 @@ def lib() -> ctypes.CDLL:
                                 ctypes.c_int, vp, ctypes.c_int, i64p, vp, vp]
     L.sage_debug_qk_int32.argtypes = [P(SageProblem), vp, vp, ctypes.c_int, ctypes.c_int, vp, vp]
     L.sage_poll_device_status.argtypes = [vp]
+    L.sage_debug_watchdog_selftest.argtypes = [ctypes.c_uint, vp]
     L.sage_attn_host.argtypes = [P(SageProblem), ctypes.c_int, vp, vp, vp, vp, ctypes.c_int,
                                  ctypes.c_float, ctypes.c_int, ctypes.c_int, vp, sz, vp]
     L.sage_host_workspace_bytes.argtypes = [P(SageProblem), ctypes.c_int, ctypes.c_int]

@@ -23,7 +23,8 @@ import torch
 from . import _lib as L
 
 __all__ = ["Problem", "Quantized", "quant_qk", "quant_qk_noalloc", "quant_v", "attn_fwd",
-           "sageattn", "sageattn_host", "debug_qk_int32", "poll_device_status"]
+           "sageattn", "sageattn_host", "debug_qk_int32", "debug_watchdog_selftest",
+           "poll_device_status"]
 
 _IN_DTYPES = {torch.float16: L.SAGE_FP16, torch.bfloat16: L.SAGE_BF16}
 # INT8 scale granularity of Q and K: "block" (128-token Q / 64-token K blocks, the
@@ -305,6 +306,13 @@ def debug_qk_int32(z: Quantized, seq: int, head_q: int) -> torch.Tensor:
                                      _ptr(s), _stream())
     L.check("sage_debug_qk_int32", st)
     return s
+
+
+def debug_watchdog_selftest(limit_us: int = 2000) -> None:
+    """Test hook: enqueue a kernel whose bounded wait runs out after limit_us and
+    records a timeout in the device watchdog word (read with poll_device_status)."""
+    L.check("sage_debug_watchdog_selftest",
+            L.lib().sage_debug_watchdog_selftest(int(limit_us), _stream()))
 
 
 def poll_device_status() -> int:

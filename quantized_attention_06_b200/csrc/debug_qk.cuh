@@ -77,4 +77,22 @@ debug_qk_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   }
 }
 
+// Failure-path self-test: thread 0 waits on an mbarrier phase that never completes
+// (its count is 1 and nothing arrives), polling as the kernels' bounded waits do, and
+// records a timeout in the watchdog word once limit_ns have passed.
+__global__ void __launch_bounds__(32) watchdog_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  fence_barrier_init();
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(b, 0)) {
+    if (global_timer_ns() - t0 > limit_ns) {
+      watchdog_trip(0x7E57);
+      return;
+    }
+  }
+}
+
 }  // namespace sage

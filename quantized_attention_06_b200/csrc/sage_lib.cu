@@ -380,6 +380,15 @@ sage_status_t sage_debug_qk_int32(const sage_problem_t* p, const int8_t* q8, con
   return launched();
 }
 
+sage_status_t sage_debug_watchdog_selftest(unsigned int limit_us, sage_stream_t stream) {
+  if (limit_us == 0 || limit_us > 1000000u) return SAGE_ERR_INVALID_ARGUMENT;
+  sage_status_t st = device_ok();
+  if (st != SAGE_OK) return st;
+  watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_us) * 1000ull);
+  return launched();
+}
+
 sage_status_t sage_poll_device_status(sage_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return SAGE_ERR_CUDA;

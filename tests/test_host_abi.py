@@ -180,3 +180,8 @@ def test_python_problem_granularity():
     assert api.Problem(1, 2, 2, 300, 64, torch.float16).k_block == 64
     with pytest.raises(ValueError):
         api.Problem(1, 2, 2, 300, 64, torch.float16, granularity="warp")
+
+
+def test_watchdog_selftest_argument_range(lib):
+    assert lib.sage_debug_watchdog_selftest(0, None) == L.SAGE_ERR_INVALID_ARGUMENT
+    assert lib.sage_debug_watchdog_selftest(1000001, None) == L.SAGE_ERR_INVALID_ARGUMENT
