@@ -19,13 +19,13 @@ What it computes, stage by stage, for one (sequence, query head) with its KV hea
    block, then added into the running output: two-level accumulation
    (vibecrowd page, How it works; heatdrop review, Key highlights).
 
-Everything after the integer scores is done in float64, with one exception
-kept apart in ``attention_head_kernel_precision``: P8 is an integer code decided
-by floating point, so for GPU parity that decision is taken with the kernel's
-own fp32 steps (fp32 logits and running max, t = fma(S, ck, log2 448 - m'),
-the documented fp32 exp2 algorithm, e4m3 rounding); the row sum l adds the same
-unrounded p, and the sums, rescale factors, PV and the output stay fp64.
-``attention_head`` is the all-fp64 definition.
+Everything after the integer scores is done in float64: ``attention_head`` is
+that all-fp64 definition and the reference every GPU parity check compares with.
+``attention_head_fp32_logits`` is a second, diagnostic path: it forms the logits,
+the running max and the exponent argument t with the fp32 operations the kernel
+uses, and then takes 2^t correctly rounded to fp32 (an fp64 exp2 followed by one
+rounding), so it shows how much of a difference comes from fp32 logits alone.
+Neither path contains any approximation of the exponential.
 
 Readings where the pages are silent:
 
@@ -39,6 +39,9 @@ Readings where the pages are silent:
 * Online-softmax block T = 128 keys.  P8 = e4m3(448 * exp(x - m')) with m' the
   running max after the block; the running sum l adds the unquantized exp values.
 * Output o = O * sv / (448 * l); lse = m + ln(l) (natural log of sum exp(x)).
+* 16-bit PV option (vibecrowd page, How it works: "FP16/FP8 for PV"): with
+  ``pv="fp16"`` or ``pv="bf16"`` V keeps its input values (no V quantization, sv = 1)
+  and P~ is rounded to that 16-bit type with scale 1; the output is O / l.
 * GQA: query head h reads KV head h // (Hq / Hkv).  Varlen: every packed
   sequence is an independent problem (its own mean, blocks and causal diagonal).
 * Causal (equal query and key lengths): key j is masked for query i when j > i.
@@ -62,9 +65,9 @@ __all__ = [
     "k_channel_mean", "smooth_k", "quantize_int8_blocks", "quantize_v_e4m3",
     "integer_scores", "online_softmax_pv", "attention_head", "sage_attention",
     "reference_attention", "attention_weights",
-    "LOG2E_F32", "LOG2_448_F32", "EXP2_COEF_F32", "EXP2_MAX_REL_ERR", "fma_f32", "exp2_f32",
-    "kernel_scale_log2",
-    "online_softmax_pv_fp32_decision", "attention_head_kernel_precision",
+    "PV_FORMATS", "round_pv", "p_scale",
+    "LOG2E_F32", "fma_f32", "exp2_rn_f32", "kernel_scale_log2",
+    "online_softmax_pv_fp32_decision", "attention_head_fp32_logits",
 ]
 
 BLKQ = 128        # tokens per Q quantization block
@@ -131,6 +134,28 @@ def e4m3_encode(values) -> np.ndarray:
                   np.rint(a / 2.0 ** -9))
     code = sign | (ef.astype(np.int64) << 3) | mf.astype(np.int64)
     return code.astype(np.uint8)
+
+
+# P (and, for the 16-bit option, V) formats of the PV product
+PV_FORMATS = ("e4m3", "fp16", "bf16")
+
+
+def p_scale(pv: str) -> float:
+    """Static scale of P~ (<= 1) before rounding: 448 fills e4m3; 16-bit types take P~ as is."""
+    if pv not in PV_FORMATS:
+        raise ValueError(f"pv must be one of {PV_FORMATS}, got {pv!r}")
+    return P_SCALE if pv == "e4m3" else 1.0
+
+
+def round_pv(x, pv: str) -> np.ndarray:
+    """Round P values to the PV operand format (e4m3 satfinite, fp16 or bf16; RNE)."""
+    if pv == "e4m3":
+        return e4m3_round(x)
+    if pv == "fp16":
+        return round_binary(x, p=11, emin=-14)
+    if pv == "bf16":
+        return round_binary(x, p=8, emin=-126)
+    raise ValueError(f"pv must be one of {PV_FORMATS}, got {pv!r}")
 
 
 # --------------------------------------------------------------------------
@@ -202,16 +227,19 @@ def integer_scores(q8: np.ndarray, k8: np.ndarray) -> np.ndarray:
 # --------------------------------------------------------------------------
 
 def online_softmax_pv(x_rows: np.ndarray, vvals: np.ndarray, sv: np.ndarray,
-                      quantize_p: bool = True):
+                      quantize_p: bool = True, pv: str = "e4m3"):
     """Online softmax over KV blocks of KV_TILE keys with two-level PV accumulation.
 
     x_rows: (r, n_kv) float64 logits, already dequantized and scaled, with masked
     entries set to -inf.  vvals: (n_kv, d) float64 V values (e4m3 values when
-    quantized).  sv: (d,) per-channel V scales (ones when not quantized).
+    quantized, the input values for a 16-bit ``pv``).  sv: (d,) per-channel V
+    scales (ones when V is not quantized).  ``pv`` names the format P is rounded
+    to (``round_pv``) at its static scale (``p_scale``).
     Returns (out (r, d), lse (r,)).
     """
     r, n_kv = x_rows.shape
     d = vvals.shape[1]
+    ps = p_scale(pv)
     m = np.full(r, -np.inf)
     l = np.zeros(r)
     o = np.zeros((r, d))
@@ -224,18 +252,18 @@ def online_softmax_pv(x_rows: np.ndarray, vvals: np.ndarray, sv: np.ndarray,
         p = np.where(live[:, None], np.exp(x - m_safe[:, None]), 0.0)
         alpha = np.where(np.isfinite(m), np.exp(m - m_safe), 0.0)
         l = l * alpha + np.sum(p, axis=1)
-        p8 = e4m3_round(P_SCALE * p) if quantize_p else P_SCALE * p
-        pv_blk = p8 @ vvals[t0:t0 + KV_TILE]          # first level: one KV block
+        pq = round_pv(ps * p, pv) if quantize_p else ps * p
+        pv_blk = pq @ vvals[t0:t0 + KV_TILE]           # first level: one KV block
         o = o * alpha[:, None] + pv_blk                # second level: running output
         m = np.where(live, m_new, m)
-    out = o * sv[None, :] / (P_SCALE * l[:, None])
+    out = o * sv[None, :] / (ps * l[:, None])
     lse = m + np.log(l)
     return out, lse
 
 
 def attention_head(q, k, v, *, causal: bool = False, sm_scale: float | None = None,
                    rows=None, quantize: bool = True, smooth: bool = True,
-                   qblk: int = BLKQ, kblk: int = BLKK) -> dict:
+                   qblk: int = BLKQ, kblk: int = BLKK, pv: str = "e4m3") -> dict:
     """Quantized attention for one (sequence, query head) with its KV head.
 
     q: (n, d), k, v: (n_kv, d), float32 holding the input values.  ``rows`` picks a
@@ -243,7 +271,9 @@ def attention_head(q, k, v, *, causal: bool = False, sm_scale: float | None = No
     ``quantize=False`` replaces every quantizer by the identity (fp64 values,
     P unrounded), which reduces the method to exact softmax attention.  qblk / kblk
     are the INT8 scale blocks of Q and K in tokens (128 / 64 as the method states;
-    1 / 32 for the per-thread granularity).
+    1 / 32 for the per-thread granularity).  ``pv`` is the PV format: "e4m3" (the
+    method: e4m3 P and per-channel e4m3 V) or "fp16" / "bf16" (P rounded to that
+    type, V at its input values).
     """
     q = np.asarray(q, dtype=np.float32)
     k = np.asarray(k, dtype=np.float32)
@@ -261,14 +291,20 @@ def attention_head(q, k, v, *, causal: bool = False, sm_scale: float | None = No
         ks = smooth_k(k, mu)
         q8, sq = quantize_int8_blocks(q, qblk)
         k8, sk = quantize_int8_blocks(ks, kblk)
-        v8, sv = quantize_v_e4m3(v)
         s_int = integer_scores(q8[rows], k8[:n_kv])
         row_scale = sq[rows // qblk].astype(np.float64)
         col_scale = sk[np.arange(n_kv) // kblk].astype(np.float64)
         x = s_int.astype(np.float64) * row_scale[:, None] * col_scale[None, :] * scale
-        vvals = e4m3_decode(v8)
-        svv = sv.astype(np.float64)
-        res.update(q8=q8, q_scale=sq, k8=k8, k_scale=sk, v8=v8, v_scale=sv, s_int=s_int)
+        res.update(q8=q8, q_scale=sq, k8=k8, k_scale=sk, s_int=s_int)
+        if pv == "e4m3":
+            v8, sv = quantize_v_e4m3(v)
+            vvals = e4m3_decode(v8)
+            svv = sv.astype(np.float64)
+            res.update(v8=v8, v_scale=sv)
+        else:
+            p_scale(pv)                                 # validates the format name
+            vvals = v.astype(np.float64)
+            svv = np.ones(d)
     else:
         ks = np.asarray(k, dtype=np.float64) - mu.astype(np.float64)[None, :]
         x = (q[rows].astype(np.float64) @ ks.T) * scale
@@ -276,7 +312,7 @@ def attention_head(q, k, v, *, causal: bool = False, sm_scale: float | None = No
         svv = np.ones(d)
     if causal:
         x = np.where(np.arange(n_kv)[None, :] > rows[:, None], -np.inf, x)
-    out, lse = online_softmax_pv(x, vvals, svv, quantize_p=quantize)
+    out, lse = online_softmax_pv(x, vvals, svv, quantize_p=quantize, pv=pv)
     res.update(out=out, lse=lse, rows=rows)
     return res
 
@@ -307,7 +343,8 @@ def attention_weights(q, k, *, causal=False, sm_scale=None, quantize=True, smoot
 
 
 def sage_attention(q, k, v, *, causal=False, sm_scale=None, cu_seqlens=None,
-                   quantize=True, smooth=True, qblk: int = BLKQ, kblk: int = BLKK) -> np.ndarray:
+                   quantize=True, smooth=True, qblk: int = BLKQ, kblk: int = BLKK,
+                   pv: str = "e4m3") -> np.ndarray:
     """Whole-batch quantized attention in float64.
 
     Dense: q (B,Hq,N,d), k, v (B,Hkv,N,d) -> out (B,Hq,N,d).
@@ -321,7 +358,7 @@ def sage_attention(q, k, v, *, causal=False, sm_scale=None, cu_seqlens=None,
             for h in range(Hq):
                 out[b, h] = attention_head(q[b, h], k[b, h // g], v[b, h // g], causal=causal,
                                            sm_scale=sm_scale, quantize=quantize,
-                                           smooth=smooth, qblk=qblk, kblk=kblk)["out"]
+                                           smooth=smooth, qblk=qblk, kblk=kblk, pv=pv)["out"]
         return out
     T, Hq, d = q.shape
     g = Hq // k.shape[1]
@@ -330,7 +367,7 @@ def sage_attention(q, k, v, *, causal=False, sm_scale=None, cu_seqlens=None,
         for h in range(Hq):
             out[s0:s1, h] = attention_head(q[s0:s1, h], k[s0:s1, h // g], v[s0:s1, h // g],
                                            causal=causal, sm_scale=sm_scale, quantize=quantize,
-                                           smooth=smooth, qblk=qblk, kblk=kblk)["out"]
+                                           smooth=smooth, qblk=qblk, kblk=kblk, pv=pv)["out"]
     return out
 
 
@@ -349,23 +386,16 @@ def reference_attention(q, k, v, *, causal=False, sm_scale=None) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
-# The P8 decision taken in the kernel's precision
+# fp32 logits with a correctly rounded exponential (diagnostic path)
 # --------------------------------------------------------------------------
-# P8 is an integer code decided by floating point, so for parity both sides take
-# that decision with the same fp32 arithmetic: logits u = S * ck in the log2
-# domain, the running max m' over 64-key halves, t = fma(S, ck, log2(448) - m'),
-# and 2^t by the documented exp2 algorithm below.  Everything else (the running
-# sum l, the rescale factors, PV and the output) stays in fp64.
+# The kernel forms the logits in fp32: u = S * ck in the log2 domain with
+# ck = fp32(fp32(q_scale * k_scale) * fp32(sm_scale * log2 e)), the running max m'
+# as the fp32 max over K blocks of (largest score * block factor), and the exponent
+# argument t = fma(S, ck, log2(P scale) - m').  This path takes exactly those fp32
+# steps and then 2^t correctly rounded to fp32; everything else (the running sum l,
+# the rescale factors, PV and the output) is fp64, as in ``attention_head``.
 
 LOG2E_F32 = np.float32(1.4426950408889634)
-LOG2_448_F32 = np.float32(8.807354922057604)
-MAGIC_F32 = np.float32(12582912.0)           # 1.5 * 2^23
-# 1 + c1 f + c2 f^2: minimal relative error for 2^f on [-1/2, 1/2] with the constant
-# term fixed at 1 (integer t then gives exact powers of two); max relative error
-# 1.97e-3, far below the e4m3 step of P (6.25% to 12.5%)
-EXP2_COEF_F32 = tuple(np.array([0x3F800000, 0x3F33F42F, 0x3E759F88],
-                               dtype=np.uint32).view(np.float32))
-EXP2_MAX_REL_ERR = 1.97e-3
 
 
 def fma_f32(a, b, c) -> np.ndarray:
@@ -393,19 +423,15 @@ def fma_f32(a, b, c) -> np.ndarray:
     return r.astype(np.float32)
 
 
-def exp2_f32(t) -> np.ndarray:
-    """2^t in fp32 operations: r = t + 1.5*2^23 rounds t to n = rint(t) (magic-number
-    rounding), f = t - (r - 1.5*2^23) in [-1/2, 1/2], Horner polynomial
-    1 + c1 f + c2 f^2 (fp32 FMAs), and n, clamped below at -125 so the result
-    stays a normal number, added to the exponent field."""
-    t = np.asarray(t, dtype=np.float32)
-    r = (t + MAGIC_F32).astype(np.float32)
-    n = np.maximum(r.view(np.int32), np.int32(0x4B400000 - 125)) - np.int32(0x4B400000)
-    f = (t - (r - MAGIC_F32).astype(np.float32)).astype(np.float32)
-    c0, c1, c2 = EXP2_COEF_F32
-    p = fma_f32(c2, f, c1)
-    p = fma_f32(p, f, c0)
-    return (p.view(np.int32) + (n << 23)).view(np.float32)
+def exp2_rn_f32(t) -> np.ndarray:
+    """2^t for fp32 t, rounded once to fp32 (round to nearest even).
+
+    np.exp2 in float64 is accurate to about one fp64 ulp, 2^-29 of an fp32 ulp, so
+    the single rounding to fp32 is the correctly rounded result except for
+    arguments whose exact power lies within that distance of an fp32 midpoint.
+    """
+    with np.errstate(over="ignore"):          # 2^t beyond the fp32 range rounds to inf
+        return np.exp2(np.asarray(t, dtype=np.float32).astype(np.float64)).astype(np.float32)
 
 
 def kernel_scale_log2(d: int, sm_scale: float | None = None) -> np.float32:
@@ -415,18 +441,21 @@ def kernel_scale_log2(d: int, sm_scale: float | None = None) -> np.float32:
 
 
 def online_softmax_pv_fp32_decision(s_int, sq_rows, sk_blocks, scale_log2, valid, vvals, sv,
-                                    quantize_p: bool = True, kblk: int = BLKK):
-    """Online softmax with the P8 codes decided in the kernel's fp32 precision.
+                                    quantize_p: bool = True, kblk: int = BLKK,
+                                    pv: str = "e4m3"):
+    """Online softmax with fp32 logits and running max and an exact fp32 2^t.
 
     s_int: (r, n_kv) exact scores; sq_rows: (r,) float32 Q scales; sk_blocks:
     float32 K scales per kblk-key block; scale_log2: float32 sm_scale*log2(e);
     valid: (r, n_kv) bool key mask; vvals (n_kv, d) and sv (d,) as in
-    online_softmax_pv.  The running max m' is the fp32 max of fp32 products of
-    each K block's largest score with that block's scale factor.
+    online_softmax_pv; ``pv`` the PV format.  The running max m' is the fp32 max
+    of fp32 products of each K block's largest score with that block's factor.
     Returns (out, lse).
     """
     r, n_kv = s_int.shape
     d = vvals.shape[1]
+    ps = p_scale(pv)
+    log2_ps = np.float32(math.log2(ps))
     per_tile = KV_TILE // kblk
     nblk = per_tile * (-(-n_kv // KV_TILE))
     skb = np.zeros(nblk, dtype=np.float32)
@@ -439,12 +468,12 @@ def online_softmax_pv_fp32_decision(s_int, sq_rows, sk_blocks, scale_log2, valid
         cols = np.arange(t0, min(n_kv, t0 + KV_TILE))
         S = s_int[:, cols].astype(np.int64)
         ok = valid[:, cols]
-        half = (cols - t0) // kblk                                                 # K block in tile
+        blk = (cols - t0) // kblk                                                  # K block in tile
         ck = np.stack([((sq_rows * skb[per_tile * j + h]).astype(np.float32) * scale_log2).astype(np.float32)
                        for h in range(per_tile)], axis=1)                          # (r, per_tile)
         mt = np.full(r, -np.inf, dtype=np.float32)
         for h in range(per_tile):
-            sel = half == h
+            sel = blk == h
             if not np.any(sel):
                 continue
             Sh = np.where(ok[:, sel], S[:, sel], np.iinfo(np.int64).min)
@@ -453,32 +482,28 @@ def online_softmax_pv_fp32_decision(s_int, sq_rows, sk_blocks, scale_log2, valid
             prod = (imax.astype(np.float32) * ck[:, h]).astype(np.float32)
             mt = np.maximum(mt, np.where(has, prod, np.float32(-np.inf)))
         m_new = np.maximum(m32, mt)
-        nbias = (LOG2_448_F32 - m_new).astype(np.float32)
-        ckc = ck[:, half]                                                          # (r, T)
-        tt = fma_f32(S.astype(np.float32), ckc, nbias[:, None])
-        p = np.where(ok, exp2_f32(tt).astype(np.float64), 0.0)
-        p8 = e4m3_round(p) if quantize_p else p
-        # fp64 accumulation in the frame of the fp32 running max (log2 domain); the row
-        # sum takes the same unrounded p whose e4m3 codes feed PV, so the exp2
-        # approximation enters the numerator and the denominator alike
+        nbias = (log2_ps - m_new).astype(np.float32)
+        tt = fma_f32(S.astype(np.float32), ck[:, blk], nbias[:, None])
+        p = np.where(ok, exp2_rn_f32(tt).astype(np.float64), 0.0)                   # ps * P~
+        pq = round_pv(p, pv) if quantize_p else p
         alpha = np.where(np.isfinite(m32), np.exp2(m32.astype(np.float64) - m_new.astype(np.float64)), 0.0)
         l = l * alpha + np.sum(p, axis=1)
-        o = o * alpha[:, None] + p8 @ vvals[cols]
+        o = o * alpha[:, None] + pq @ vvals[cols]
         m32 = m_new
     out = o * sv[None, :] / l[:, None]
-    lse = m32.astype(np.float64) * math.log(2.0) + np.log(l / P_SCALE)
+    lse = m32.astype(np.float64) * math.log(2.0) + np.log(l / ps)
     return out, lse
 
 
-def attention_head_kernel_precision(q, k, v, *, causal=False, sm_scale=None, rows=None,
-                                    quantize_p: bool = True, qblk: int = BLKQ,
-                                    kblk: int = BLKK) -> dict:
-    """attention_head with the P8 codes decided in the kernel's fp32 precision.
+def attention_head_fp32_logits(q, k, v, *, causal=False, sm_scale=None, rows=None,
+                               quantize_p: bool = True, qblk: int = BLKQ,
+                               kblk: int = BLKK, pv: str = "e4m3") -> dict:
+    """attention_head with fp32 logits, fp32 running max and a correctly rounded 2^t.
 
     Quantization of Q, K, V and the integer scores are the same exact stages as
-    attention_head; p = 448 * 2^t comes from the fp32 logits and exp2 algorithm above,
-    P8 = e4m3(p), and the row sum l (of the unrounded p), the rescale factors, PV and
-    the output are fp64.
+    attention_head; p = P scale * P~ is fp32(2^t) with t from the kernel's fp32
+    logit steps, P = round_pv(p), and the row sum l (of the unrounded p), the
+    rescale factors, PV and the output are fp64.
     """
     q = np.asarray(q, dtype=np.float32)
     k = np.asarray(k, dtype=np.float32)
@@ -491,13 +516,19 @@ def attention_head_kernel_precision(q, k, v, *, causal=False, sm_scale=None, row
     mu = k_channel_mean(k)
     q8, sq = quantize_int8_blocks(q, qblk)
     k8, sk = quantize_int8_blocks(smooth_k(k, mu), kblk)
-    v8, sv = quantize_v_e4m3(v)
     s_int = integer_scores(q8[rows], k8[:n_kv])
     valid = np.ones((len(rows), n_kv), dtype=bool)
     if causal:
         valid = np.arange(n_kv)[None, :] <= rows[:, None]
+    res = dict(rows=rows, k_mean=mu, q8=q8, q_scale=sq, k8=k8, k_scale=sk, s_int=s_int)
+    if pv == "e4m3":
+        v8, sv = quantize_v_e4m3(v)
+        vvals, svv = e4m3_decode(v8), sv.astype(np.float64)
+        res.update(v8=v8, v_scale=sv)
+    else:
+        vvals, svv = v.astype(np.float64), np.ones(d)
     out, lse = online_softmax_pv_fp32_decision(
-        s_int, sq[rows // qblk], sk, kernel_scale_log2(d, sm_scale), valid,
-        e4m3_decode(v8), sv.astype(np.float64), quantize_p=quantize_p, kblk=kblk)
-    return dict(out=out, lse=lse, rows=rows, k_mean=mu, q8=q8, q_scale=sq, k8=k8, k_scale=sk,
-                v8=v8, v_scale=sv, s_int=s_int)
+        s_int, sq[rows // qblk], sk, kernel_scale_log2(d, sm_scale), valid, vvals, svv,
+        quantize_p=quantize_p, kblk=kblk, pv=pv)
+    res.update(out=out, lse=lse)
+    return res
