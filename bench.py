@@ -6,8 +6,8 @@ Workload (default): the kernel-sweep configuration at its longest length,
 B=1, H=32, N=32768, d=128, fp16, HND, non-causal, seeded synthetic inputs
 (Q, V ~ N(0,1); K ~ N(0,1) plus a per-channel offset ~ N(0, 3^2)).
 
-A step is one pass of the whole path on device-resident inputs: sage_quant_qk
-(K mean, Q/K INT8), sage_quant_v (V e4m3) and sage_attn_fwd.  TOPS =
+A step is one pass of the whole path on device-resident inputs: sage_quant_qkv
+(K mean, Q/K INT8, V e4m3 in one cooperative launch) and sage_attn_fwd.  TOPS =
 4*B*H*N^2*d / time (halved when causal).  Inputs (3 x 256 MiB) exceed the
 126 MB L2, so no flush is needed between steps.  Rank 0 prints one JSON line.
 
@@ -44,7 +44,10 @@ def parse():
     ap.add_argument("--n", type=int, default=32768)
     ap.add_argument("--causal", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=1536)
+    ap.add_argument("--cpu-rows", type=int, default=1536,
+                    help="query rows of the oracle sample (cpu_baseline and every reference step)")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the per-length / per-workload attention measurements")
     ap.add_argument("--granularity", default="block", choices=["block", "thread"],
                     help="INT8 scale granularity of Q/K: per block (the method as stated) or "
                          "per thread (a scale per Q token and per 32-token K block)")
@@ -62,7 +65,7 @@ def config(w, args, n_gpus):
             "batch": w.batch, "heads": w.heads_q, "seq_len": w.seqlen, "head_dim": w.head_dim,
             "causal": bool(args.causal), "layout": w.layout, "n_gpus": n_gpus,
             "l2": "inputs (3 x 256 MiB) larger than the 126 MB L2; no flush",
-            "step": "sage_quant_qk + sage_quant_v + sage_attn_fwd",
+            "step": "sage_quant_qkv + sage_attn_fwd",
             "granularity": getattr(args, "granularity", "block")}
 
 
@@ -75,33 +78,85 @@ def peaks():
     return 1590.0, 1400.0, 6650.0, "fallback"
 
 
-def cpu_sample(w, args, rows):
-    """Time the oracle on a bounded sample: one head's quantization plus `rows`
-    evenly spaced query rows against all keys.  Returns (TOPS, seconds, sample)."""
+# ---------------------------------------------------------------- CPU oracle baseline
+# The oracle is plain NumPy.  It is timed on all of the host's cores: a process pool
+# (started with spawn, one single-threaded worker per core) splits the sampled query
+# rows; every worker repeats the head's quantization (part of the sample) and then
+# computes its rows exactly as oracle.attention_head defines them.
+
+_POOL_HEAD = {}
+
+
+def _pool_init(q, k, v):
+    _POOL_HEAD.update(q=q, k=k, v=v)
+
+
+def _pool_rows(task):
     import oracle as orc
-    from quantized_attention_06_b200.inputs import generate
-    x = generate(w)
-    q, k, v = x["q"][0, 0], x["k"][0, 0], x["v"][0, 0]
-    sel = np.linspace(0, w.seqlen - 1, rows).astype(np.int64)
-    t0 = time.perf_counter()
-    thread = getattr(args, "granularity", "block") == "thread"
-    orc.attention_head_kernel_precision(q, k, v, causal=args.causal, rows=sel,
-                                        qblk=1 if thread else orc.BLKQ, kblk=32 if thread else orc.BLKK)
-    dt = time.perf_counter() - t0
-    n_keys = (sel + 1).sum() if args.causal else rows * w.seqlen
-    ops = 4.0 * n_keys * w.head_dim
-    sample = (f"head 0 quantization (Q, K, V) plus {rows} evenly spaced query rows against "
-              f"{'their causal prefix' if args.causal else f'all {w.seqlen} keys'}")
-    return ops / dt / 1e12, dt, sample
+    rows, causal, qblk, kblk = task
+    h = _POOL_HEAD
+    orc.attention_head(h["q"], h["k"], h["v"], causal=causal, rows=rows, qblk=qblk, kblk=kblk)
+    return len(rows)
 
 
-def threads_used():
+def cpu_model() -> str:
     try:
-        import threadpoolctl
-        info = threadpoolctl.threadpool_info()
-        return max([i.get("num_threads", 1) for i in info] + [1])
-    except Exception:
-        return 1
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def orc_blocks(args):
+    thread = getattr(args, "granularity", "block") == "thread"
+    return (1, 32) if thread else (128, 64)
+
+
+class OraclePool:
+    """A spawn-started pool of single-threaded oracle workers over one head."""
+
+    def __init__(self, w, args):
+        import multiprocessing as mp
+        from dataclasses import replace
+        from quantized_attention_06_b200.inputs import generate
+        # one head drawn with the workload's recipe and seed (timing sample only)
+        x = generate(replace(w, batch=1, heads_q=1, heads_kv=1))
+        self.q, self.k, self.v = x["q"][0, 0], x["k"][0, 0], x["v"][0, 0]
+        self.w, self.args = w, args
+        self.cores = os.cpu_count() or 1
+        for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+            os.environ[var] = "1"          # read by the spawned workers' NumPy
+        ctx = mp.get_context("spawn")
+        self.pool = ctx.Pool(self.cores, initializer=_pool_init, initargs=(self.q, self.k, self.v))
+        qb, kb = orc_blocks(args)
+        # warm the workers (imports, first quantization) before any timing
+        self.pool.map(_pool_rows, [(np.arange(1), False, qb, kb)] * self.cores)
+
+    def sample(self, rows):
+        """Time `rows` evenly spaced query rows (plus the head's quantization in every
+        worker).  Returns (TOPS, seconds, description)."""
+        w, args = self.w, self.args
+        sel = np.linspace(0, w.seqlen - 1, rows).astype(np.int64)
+        qb, kb = orc_blocks(args)
+        chunks = [c for c in np.array_split(sel, self.cores) if len(c)]
+        t0 = time.perf_counter()
+        self.pool.map(_pool_rows, [(c, bool(args.causal), qb, kb) for c in chunks])
+        dt = time.perf_counter() - t0
+        n_keys = (sel + 1).sum() if args.causal else rows * w.seqlen
+        ops = 4.0 * n_keys * w.head_dim
+        desc = (f"one head: quantization (Q, K, V; repeated by each of {len(chunks)} workers) "
+                f"plus {rows} evenly spaced query rows against "
+                f"{'their causal prefix' if args.causal else f'all {w.seqlen} keys'}, "
+                f"oracle.attention_head (fp64)")
+        return ops / dt / 1e12, dt, desc
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
 
 
 def max_over_ranks(values, device):
@@ -129,18 +184,20 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = workload(args)
+    pool = OraclePool(w, args)
     times = []
     for i in range(args.warmup + args.steps):
-        tops, dt, sample = cpu_sample(w, args, max(8, args.cpu_rows // 4))
+        tops, dt, sample = pool.sample(args.cpu_rows)
         if i >= args.warmup:
             times.append(tops)
+    pool.close()
     val = statistics.median(times)
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (P8 decision fp32)",
-            "data": "synthetic", "config": config(w, args, world),
-            "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads_used(), "kind": "oracle",
-                             "sample": sample},
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config(w, args, world),
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": pool.cores, "kind": "oracle",
+                             "sample": sample, "nproc": os.cpu_count(), "cpu_model": cpu_model()},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
@@ -203,6 +260,102 @@ class Clocks:
                 "power_w_max": max(power) if power else None}
 
 
+# ---------------------------------------------------------------- the metric's range
+# The metric spans seq 1K-32K at hd128 and the workloads of the other four configs.
+# Each point is timed on its own: inputs drawn on the device (same distributions as
+# inputs.py, seeded), quantized once, then the attention kernel alone (the kernel
+# figure, `attn`) and the whole step of three calls (`step`) are timed with CUDA
+# events around each launch.  Where the operands fit in L2, a 512 MiB buffer is
+# written between timed launches, so no launch starts with a warm L2.
+
+def _device_inputs(w, dev, seqlens=None):
+    import torch
+    g = torch.Generator(device=dev).manual_seed(1000 + w.seed)
+    if w.varlen:
+        total = int(sum(seqlens))
+        qs, ks = (total, w.heads_q, w.head_dim), (total, w.heads_kv, w.head_dim)
+    elif w.layout == "NHD":
+        qs, ks = ((w.batch, w.seqlen, w.heads_q, w.head_dim), (w.batch, w.seqlen, w.heads_kv, w.head_dim))
+    else:
+        qs, ks = ((w.batch, w.heads_q, w.seqlen, w.head_dim), (w.batch, w.heads_kv, w.seqlen, w.head_dim))
+    dt = torch.float16 if w.dtype == "fp16" else torch.bfloat16
+    q = torch.randn(qs, generator=g, device=dev)
+    k = torch.randn(ks, generator=g, device=dev)
+    v = torch.randn(ks, generator=g, device=dev)
+    if w.tail_frac > 0:
+        q = torch.where(torch.rand(qs, generator=g, device=dev) < w.tail_frac, q * w.tail_scale, q)
+        k = torch.where(torch.rand(ks, generator=g, device=dev) < w.tail_frac, k * w.tail_scale, k)
+    off_shape = [1] * k.dim()
+    off_shape[-1] = w.head_dim
+    off_shape[-2 if (w.layout == "NHD" or w.varlen) else 1] = w.heads_kv
+    k = k + torch.randn(off_shape, generator=g, device=dev) * w.k_offset_sigma
+    return q.to(dt), k.to(dt), v.to(dt)
+
+
+def measure_point(w, causal, dev, peak, pv="fp8", granularity="block", reps=10, seqlens=None):
+    import torch
+    from quantized_attention_06_b200 import api
+    q, k, v = _device_inputs(w, dev, seqlens)
+    cu = None
+    if w.varlen:
+        cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    layout = "NHD" if (w.layout == "NHD" or w.varlen) else "HND"
+    z = api.quant_qkv(q, k, v, layout, cu, granularity=granularity, pv=pv)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    operand_bytes = sum(t.numel() * t.element_size() for t in (z.q8, z.k8, z.v8))
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if operand_bytes < (256 << 20) else None
+
+    def time_it(fn):
+        ts = []
+        for i in range(3 + reps):
+            if flush is not None:
+                flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    attn_ms = time_it(lambda: api.attn_fwd(z, is_causal=causal, out=out))
+    ws = torch.empty(z.problem.sizes.workspace_qkv + 256, dtype=torch.uint8, device=dev)
+    step_ms = time_it(lambda: (api.quant_qkv(q, k, v, layout, cu, problem=z.problem, out=z, workspace=ws),
+                               api.attn_fwd(z, is_causal=causal, out=out)))
+    assert api.poll_device_status() == 0
+    ops = w.ops(causal, seqlens)
+    tops = ops / (attn_ms * 1e-3) / 1e12
+    return {"workload": w.name, "seq_len": w.seqlen, "causal": causal, "pv": pv,
+            "granularity": granularity, "attn_ms": attn_ms, "tops": tops, "frac": tops / peak,
+            "step_ms": step_ms, "step_tops": ops / (step_ms * 1e-3) / 1e12,
+            "l2": "flushed between launches" if flush is not None else "operands larger than L2"}
+
+
+def measure_metric_range(args, dev, peak):
+    from dataclasses import replace
+    import torch
+    from quantized_attention_06_b200.inputs import SWEEP_LENGTHS, WORKLOADS, sweep_workload
+    res = []
+    for n in SWEEP_LENGTHS:
+        for causal in (False, True):
+            res.append(measure_point(sweep_workload(n), causal, dev, peak))
+            torch.cuda.empty_cache()
+    res.append(measure_point(sweep_workload(32768), False, dev, peak, pv="fp16"))
+    res.append(measure_point(sweep_workload(32768), False, dev, peak, granularity="thread"))
+    for causal in (False, True):
+        res.append(measure_point(WORKLOADS["prefill"], causal, dev, peak))
+    res.append(measure_point(WORKLOADS["dit"], False, dev, peak))
+    w = WORKLOADS["gqa_varlen"]
+    lens = np.random.default_rng(w.seed).integers(w.varlen_range[0], w.varlen_range[1] + 1,
+                                                  size=w.varlen_count)
+    res.append(measure_point(replace(w, seqlen=int(lens.max())), True, dev, peak,
+                             seqlens=[int(x) for x in lens]))
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_sage(args):
     import torch
     import torch.distributed as dist
@@ -222,6 +375,8 @@ def run_sage(args):
         dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
 
     w = workload(args)
+    # the oracle's worker pool is spawned before any CUDA work (rank 0, one GPU only)
+    pool = OraclePool(w, args) if (rank == 0 and world == 1) else None
     x = generate(w)
     host = {n: torch.from_numpy(x[n]).to(torch.float16).pin_memory() for n in ("q", "k", "v")}
     del x
@@ -230,13 +385,13 @@ def run_sage(args):
     z = api.Quantized(p, "HND")
     ws_qk = torch.empty(max(1, p.sizes.workspace_qk // 8), dtype=torch.float64, device=dev)
     ws_v = torch.empty(max(1, p.sizes.workspace_v // 4), dtype=torch.float32, device=dev)
+    ws_qkv = torch.empty(p.sizes.workspace_qkv + 256, dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
-    launches_per_step = 7  # k_colsum, k_mean, quant_qk, v_colmax, v_finalize, quant_v, attn
+    launches_per_step = 2  # quant_fused (Q, K, V in one cooperative launch), attention
 
     def step(ev=None):
-        api.quant_qk(q, k, "HND", problem=p, out=z, workspace=ws_qk)
-        api.quant_v(v, z, workspace=ws_v)
+        api.quant_qkv(q, k, v, "HND", problem=p, out=z, workspace=ws_qkv)
         if ev is not None:
             ev[0].record(stream)
         api.attn_fwd(z, is_causal=args.causal, out=out)
@@ -311,6 +466,7 @@ def run_sage(args):
             torch.cuda.synchronize()
             ts.append(a.elapsed_time(b))
         return statistics.median(ts)
+    qkv_ms = timed(lambda: api.quant_qkv(q, k, v, "HND", problem=p, out=z, workspace=ws_qkv))
     qk_ms = timed(lambda: api.quant_qk(q, k, "HND", problem=p, out=z, workspace=ws_qk))
     v_ms = timed(lambda: api.quant_v(v, z, workspace=ws_v))
     elems_q = q.numel()
@@ -320,6 +476,11 @@ def run_sage(args):
 
     bf16, bf16_sus, hbm, src = peaks()
     peak = bf16 * NOMINAL_INT8_OVER_BF16
+    sweep = None
+    if not args.no_sweep:
+        del q, k, v, out, z, ws_qk, ws_v
+        torch.cuda.empty_cache()
+        sweep = measure_metric_range(args, dev, peak)
     achieved = ops / (attn_mean * 1e-3) / 1e12
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
@@ -347,6 +508,10 @@ def run_sage(args):
                          "frac_of_datasheet_4500": achieved / 4500.0},
             "e2e": e2e,
             "quant": {"unit": "GB/s", "hbm_peak": hbm,
+                      "quant_qkv": {"ms": qkv_ms,
+                                    "achieved": (qk_bytes + v_bytes) / (qkv_ms * 1e-3) / 1e9,
+                                    "frac": (qk_bytes + v_bytes) / (qkv_ms * 1e-3) / 1e9 / hbm,
+                                    "bytes": qk_bytes + v_bytes, "launches": 1},
                       "quant_qk": {"ms": qk_ms, "achieved": qk_bytes / (qk_ms * 1e-3) / 1e9,
                                    "frac": qk_bytes / (qk_ms * 1e-3) / 1e9 / hbm,
                                    "bytes": qk_bytes},
@@ -355,10 +520,14 @@ def run_sage(args):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
         }
-        if world == 1:
-            tops, dt, sample = cpu_sample(w, args, args.cpu_rows)
-            line["cpu_baseline"] = {"value": tops, "unit": UNIT, "cores": threads_used(),
-                                    "kind": "oracle", "sample": sample, "seconds": dt}
+        if sweep is not None:
+            line["sweep"] = sweep
+        if pool is not None:
+            tops, dt, sample = pool.sample(args.cpu_rows)
+            pool.close()
+            line["cpu_baseline"] = {"value": tops, "unit": UNIT, "cores": pool.cores,
+                                    "kind": "oracle", "sample": sample, "seconds": dt,
+                                    "nproc": os.cpu_count(), "cpu_model": cpu_model()}
         print(json.dumps(line))
     if world > 1:
         dist.barrier()

@@ -21,11 +21,20 @@
  *   the device watchdog word read by sage_poll_device_status(), the scratch
  *   array of sage_quant_qk_noalloc and the copy streams of sage_attn_host.
  * - Work is enqueued on `stream` (a cudaStream_t); calls return once enqueued.
+ *   The library works on the calling thread's current CUDA device: every device
+ *   pointer and `stream` must belong to it (make that device current first, e.g.
+ *   cudaSetDevice).  A stream of another device is rejected with
+ *   SAGE_ERR_INVALID_ARGUMENT; pointers cannot be checked and must not be another
+ *   device's memory.
  * - Errors: argument problems return SAGE_ERR_INVALID_ARGUMENT or
  *   SAGE_ERR_UNSUPPORTED before anything is enqueued; a failed launch returns
  *   SAGE_ERR_CUDA.  A kernel whose bounded wait runs out records
- *   SAGE_ERR_DEVICE_TIMEOUT in the watchdog word and exits early (its outputs
- *   are then undefined); the host reads that with sage_poll_device_status().
+ *   SAGE_ERR_DEVICE_TIMEOUT in the device watchdog word and exits early (its
+ *   outputs are then undefined).  The word is sticky: until
+ *   sage_poll_device_status() reads and clears it, every later kernel of the
+ *   library on that device sees it set and returns at once without writing its
+ *   outputs, while the entry points that enqueued them still return SAGE_OK.
+ *   Poll after work whose results matter.
  * - Input tensors q, k, v hold fp16 or bf16 values with a contiguous last
  *   (head_dim) dimension.  Their other three dimensions are given as element
  *   strides {stride_batch, stride_head, stride_token}: HND (B,H,N,d) and
@@ -45,8 +54,9 @@
  *   k_scale float [Hkv][T_pad/64]       one scale per 64-token block of a sequence
  *                 ([Hkv][T_pad/32], one per 32-token block, with SAGE_GRAN_THREAD)
  *   k_mean  float [B  ][Hkv][d]         per-channel mean of K over the sequence
- *   v8      uint8 [Hkv][d][T_pad]       e4m3 codes, transposed (token-contiguous)
- *   v_scale float [B  ][Hkv][d]         per-channel V scale
+ *   v8      uint8 [Hkv][d][T_pad]       e4m3 codes, transposed (token-contiguous);
+ *                 with SAGE_PV_FP16 two bytes per entry: V's own 16-bit values
+ *   v_scale float [B  ][Hkv][d]         per-channel V scale (1.0 with SAGE_PV_FP16)
  * Dequantized values: q = q8 * q_scale, k - k_mean = k8 * k_scale,
  * v = e4m3(v8) * v_scale.
  */
@@ -83,6 +93,14 @@ typedef enum { SAGE_FP16 = 0, SAGE_BF16 = 1, SAGE_FP32 = 2 } sage_dtype_t;
  *   into the same per-row, per-32-key factors. */
 typedef enum { SAGE_GRAN_BLOCK = 0, SAGE_GRAN_THREAD = 1 } sage_granularity_t;
 
+/* Format of the P V product (vibecrowd page "thu-ml--sageattention", How it works:
+ * FP16/FP8 for PV).
+ * SAGE_PV_FP8 (0, the method as stated): P and V in FP8 e4m3, V with per-channel scales.
+ * SAGE_PV_FP16 (1): the accuracy fallback.  V keeps its 16-bit input values (fp16 or
+ *   bf16, no V quantization) and P~ (<= 1) is rounded to that same type; the PV
+ *   MMA runs in that type with FP32 accumulation, two levels as with FP8. */
+typedef enum { SAGE_PV_FP8 = 0, SAGE_PV_FP16 = 1 } sage_pv_t;
+
 /* Problem description shared by all entry points. */
 typedef struct {
   int batch;              /* B: dense batch size, or number of packed sequences (<= 1024) */
@@ -94,6 +112,7 @@ typedef struct {
   const int32_t* cu_seqlens_host; /* host, NULL for dense; else [batch+1] prefix sums of the
                                      packed sequence lengths, cu[0] = 0, non-decreasing */
   sage_granularity_t granularity; /* INT8 scale granularity of Q and K (zero: per block) */
+  sage_pv_t pv;           /* format of the P V product (zero: FP8 e4m3) */
 } sage_problem_t;
 
 /* Byte sizes of the quantized buffers and of the quantization workspaces. */
@@ -102,6 +121,7 @@ typedef struct {
   size_t workspace_qk;    /* scratch needed by sage_quant_qk */
   size_t workspace_v;     /* scratch needed by sage_quant_v */
   size_t t_pad;           /* T_pad, the padded token count */
+  size_t workspace_qkv;   /* scratch needed by sage_quant_qkv */
 } sage_sizes_t;
 
 /* Fill *sizes (host) for problem *p (host).  Pure host computation. */
@@ -141,7 +161,9 @@ sage_status_t sage_quant_qk(const sage_problem_t* p,
  *   more scratch than that (sizes.workspace_qk > SAGE_NOALLOC_SCRATCH_BYTES).
  * - The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call before
- *   any stream capture.  It allocates nothing (no cudaMalloc / cudaFree).
+ *   any stream capture.  It allocates nothing (no cudaMalloc / cudaFree).  The
+ *   address is kept for the life of the process: after cudaDeviceReset() on a
+ *   device, this entry point must not be called on that device again.
  * - All calls share the array, which keeps the last call's contents (nothing in it
  *   needs clearing); calls that overlap on the GPU, from any stream or thread, race.
  */
@@ -159,10 +181,35 @@ sage_status_t sage_quant_qk_noalloc(const sage_problem_t* p,
  *   v8 = e4m3_rne_satfinite(fp32(v * fp32(448/vmax)))   (vmax == 0: sv = 0, codes 0)
  * Writes v8 and v_scale.  `workspace` must hold sizes.workspace_v bytes.
  * Launches three kernels on `stream`.
+ * With p->pv == SAGE_PV_FP16: copies V's 16-bit values into the same transposed
+ * layout (two bytes per entry) and sets v_scale to 1; no workspace is needed
+ * (sizes.workspace_v is 0 and `workspace` may be NULL).  Two launches.
  */
 sage_status_t sage_quant_v(const sage_problem_t* p, const void* v, const int64_t v_strides[3],
                            uint8_t* v8, float* v_scale, void* workspace, size_t workspace_bytes,
                            sage_stream_t stream);
+
+/*
+ * sage_quant_qkv - sage_quant_qk and sage_quant_v in one launch.
+ * (Same sources and arithmetic as those two entry points; the tutorial page
+ * "SageAttention终极指南", 源码结构解析, places quantization in its own module.)
+ * Writes q8, q_scale, k8, k_scale, k_mean, v8 and v_scale exactly as the two separate
+ * calls would: every code, scale and mean is bit-identical.  One cooperative,
+ * persistent launch (one CTA per SM): Q is quantized while the K sums and V maxima
+ * are gathered, a grid-wide barrier precedes the means and V scales, another precedes
+ * the K and V codes.  Tiles move by TMA, so besides the rules for every entry point
+ * the smallest of the three element strides of each input must be at least
+ * head_dim (rows do not overlap); SAGE_ERR_INVALID_ARGUMENT otherwise.
+ * `workspace` must hold sizes.workspace_qkv bytes; its contents on entry do not
+ * matter.  SAGE_ERR_UNSUPPORTED if the device cannot launch cooperative kernels.
+ */
+sage_status_t sage_quant_qkv(const sage_problem_t* p,
+                             const void* q, const int64_t q_strides[3],
+                             const void* k, const int64_t k_strides[3],
+                             const void* v, const int64_t v_strides[3],
+                             int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
+                             float* k_mean, void* v8, float* v_scale, void* workspace,
+                             size_t workspace_bytes, sage_stream_t stream);
 
 /*
  * sage_attn_fwd - the attention kernel (tcgen05 INT8 QK^T and FP8 PV, TMEM accumulators).
@@ -175,6 +222,10 @@ sage_status_t sage_quant_v(const sage_problem_t* p, const void* v, const int64_t
  *   m'   = max(m, max_j x_j);   P~_j = exp(x_j - m');   l = l e^{m-m'} + sum_j P~_j
  *   P8   = e4m3(448 P~);  PV_blk = P8 V8 (FP32, fresh per block);  O = O e^{m-m'} + PV_blk
  *   out  = O * v_scale / (448 l)           lse = m + ln(l)   (natural log)
+ *   (SAGE_PV_FP16: P = P~ rounded to the input's 16-bit type, PV_blk = P V16,
+ *    out = O / l.)
+ * The logits, the running max and the exponent argument are formed in fp32 and
+ * exp is the hardware base-2 exponential (within 2 ulp of exact).
  * sm_scale <= 0 selects 1/sqrt(head_dim).  is_causal != 0 applies the mask above.
  * out: written in out_dtype (SAGE_FP16, SAGE_BF16 or SAGE_FP32) with element
  * strides out_strides {batch, head, token}, last dimension contiguous, the

@@ -20,11 +20,13 @@ NOALLOC_SCRATCH_BYTES = 8 << 20  # SAGE_NOALLOC_SCRATCH_BYTES
 
 SAGE_FP16, SAGE_BF16, SAGE_FP32 = 0, 1, 2
 SAGE_GRAN_BLOCK, SAGE_GRAN_THREAD = 0, 1
+SAGE_PV_FP8, SAGE_PV_FP16 = 0, 1
 
 EXPORTS = (
     "sage_buffer_sizes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd",
     "sage_debug_qk_int32", "sage_poll_device_status", "sage_quant_qk_noalloc",
     "sage_attn_host", "sage_host_workspace_bytes", "sage_debug_watchdog_selftest",
+    "sage_quant_qkv",
     "sage_status_string",
 )
 
@@ -39,13 +41,14 @@ class SageProblem(ctypes.Structure):
         ("dtype", ctypes.c_int),
         ("cu_seqlens_host", ctypes.POINTER(ctypes.c_int32)),
         ("granularity", ctypes.c_int),  # SAGE_GRAN_BLOCK / SAGE_GRAN_THREAD
+        ("pv", ctypes.c_int),           # SAGE_PV_FP8 / SAGE_PV_FP16
     ]
 
 
 class SageSizes(ctypes.Structure):
     _fields_ = [(name, ctypes.c_size_t) for name in (
         "q8", "q_scale", "k8", "k_scale", "k_mean", "v8", "v_scale",
-        "workspace_qk", "workspace_v", "t_pad")]
+        "workspace_qk", "workspace_v", "t_pad", "workspace_qkv")]
 
 
 class SageError(RuntimeError):
@@ -72,6 +75,8 @@ def lib() -> ctypes.CDLL:
     L.sage_buffer_sizes.argtypes = [P(SageProblem), P(SageSizes)]
     L.sage_quant_qk.argtypes = [P(SageProblem), vp, i64p, vp, i64p, vp, vp, vp, vp, vp, vp, sz, vp]
     L.sage_quant_v.argtypes = [P(SageProblem), vp, i64p, vp, vp, vp, sz, vp]
+    L.sage_quant_qkv.argtypes = [P(SageProblem), vp, i64p, vp, i64p, vp, i64p, vp, vp, vp, vp, vp,
+                                 vp, vp, vp, sz, vp]
     L.sage_quant_qk_noalloc.argtypes = [P(SageProblem), vp, i64p, vp, i64p, vp, vp, vp, vp, vp, vp]
     L.sage_attn_fwd.argtypes = [P(SageProblem), vp, vp, vp, vp, vp, vp, ctypes.c_float,
                                 ctypes.c_int, vp, ctypes.c_int, i64p, vp, vp]

@@ -22,7 +22,7 @@ import torch
 
 from . import _lib as L
 
-__all__ = ["Problem", "Quantized", "quant_qk", "quant_qk_noalloc", "quant_v", "attn_fwd",
+__all__ = ["Problem", "Quantized", "quant_qk", "quant_qk_noalloc", "quant_v", "quant_qkv", "attn_fwd",
            "sageattn", "sageattn_host", "debug_qk_int32", "debug_watchdog_selftest",
            "poll_device_status"]
 
@@ -31,6 +31,9 @@ _IN_DTYPES = {torch.float16: L.SAGE_FP16, torch.bfloat16: L.SAGE_BF16}
 # method as stated) or "thread" (a scale per Q token and per 32-token K block)
 _GRANULARITY = {"block": L.SAGE_GRAN_BLOCK, "thread": L.SAGE_GRAN_THREAD}
 _OUT_DTYPES = {torch.float16: L.SAGE_FP16, torch.bfloat16: L.SAGE_BF16, torch.float32: L.SAGE_FP32}
+# format of the P V product: "fp8" (e4m3 P and V, the method as stated) or "fp16" (P and V
+# in the input's 16-bit type, the accuracy fallback)
+_PV = {"fp8": L.SAGE_PV_FP8, "fp16": L.SAGE_PV_FP16}
 
 
 def _ptr(t) -> int | None:
@@ -45,12 +48,15 @@ class Problem:
     """Shapes of one attention call (sage_problem_t)."""
 
     def __init__(self, batch, heads_q, heads_kv, seqlen, head_dim, dtype, cu_seqlens=None,
-                 granularity="block"):
+                 granularity="block", pv="fp8"):
         if dtype not in _IN_DTYPES:
             raise TypeError(f"q/k/v must be float16 or bfloat16, got {dtype}")
         if granularity not in _GRANULARITY:
             raise ValueError(f"granularity must be 'block' or 'thread', got {granularity!r}")
+        if pv not in _PV:
+            raise ValueError(f"pv must be 'fp8' or 'fp16', got {pv!r}")
         self.granularity = granularity
+        self.pv = pv
         self.dtype = dtype
         self.varlen = cu_seqlens is not None
         if self.varlen:
@@ -64,7 +70,7 @@ class Problem:
             self.cu_list = None
             cu_ptr = ctypes.POINTER(ctypes.c_int32)()
         self.c = L.SageProblem(batch, heads_q, heads_kv, seqlen, head_dim, _IN_DTYPES[dtype], cu_ptr,
-                               _GRANULARITY[granularity])
+                               _GRANULARITY[granularity], _PV[pv])
         self.batch, self.heads_q, self.heads_kv = batch, heads_q, heads_kv
         self.seqlen, self.head_dim = seqlen, head_dim
         sz = L.SageSizes()
@@ -81,11 +87,12 @@ class Problem:
         return 32 if self.granularity == "thread" else 64
 
     @staticmethod
-    def from_tensors(q, k, tensor_layout="HND", cu_seqlens=None, granularity="block") -> "Problem":
+    def from_tensors(q, k, tensor_layout="HND", cu_seqlens=None, granularity="block",
+                     pv="fp8") -> "Problem":
         if cu_seqlens is not None:
             _, hq, d = q.shape
             hkv = k.shape[1]
-            return Problem(0, hq, hkv, 0, d, q.dtype, cu_seqlens, granularity)
+            return Problem(0, hq, hkv, 0, d, q.dtype, cu_seqlens, granularity, pv)
         if tensor_layout == "HND":
             b, hq, n, d = q.shape
             hkv = k.shape[1]
@@ -94,7 +101,7 @@ class Problem:
             hkv = k.shape[2]
         else:
             raise ValueError(f"tensor_layout must be 'HND' or 'NHD', got {tensor_layout!r}")
-        return Problem(b, hq, hkv, n, d, q.dtype, granularity=granularity)
+        return Problem(b, hq, hkv, n, d, q.dtype, granularity=granularity, pv=pv)
 
 
 def _strides(t: torch.Tensor, tensor_layout: str, varlen: bool):
@@ -131,13 +138,22 @@ def _require_cuda(*ts):
     for t in ts:
         if not (isinstance(t, torch.Tensor) and t.is_cuda):
             raise RuntimeError("sage kernels need CUDA tensors on a B200; there is no CPU fallback")
+    dev = ts[0].device
+    if any(t.device != dev for t in ts):
+        raise ValueError("all tensors of one call must be on the same CUDA device")
+    return dev
 
 
 def quant_qk(q, k, tensor_layout="HND", cu_seqlens=None, problem=None, out: Quantized = None,
-             workspace=None, granularity="block") -> Quantized:
-    """K smoothing + per-block INT8 quantization of Q and K (sage_quant_qk)."""
-    _require_cuda(q, k)
-    p = problem or Problem.from_tensors(q, k, tensor_layout, cu_seqlens, granularity)
+             workspace=None, granularity="block", pv="fp8") -> Quantized:
+    """K smoothing + per-block INT8 quantization of Q and K (sage_quant_qk).
+    ``pv`` fixes the PV format of the attention call that follows ("fp8" or "fp16")."""
+    with torch.cuda.device(_require_cuda(q, k)):
+        return _quant_qk(q, k, tensor_layout, cu_seqlens, problem, out, workspace, granularity, pv)
+
+
+def _quant_qk(q, k, tensor_layout, cu_seqlens, problem, out, workspace, granularity, pv):
+    p = problem or Problem.from_tensors(q, k, tensor_layout, cu_seqlens, granularity, pv)
     z = out or Quantized(p, tensor_layout)
     dev = q.device
     sz = p.sizes
@@ -165,7 +181,11 @@ def quant_qk_noalloc(q, k, tensor_layout="HND", cu_seqlens=None, problem=None,
     allocate device memory when they quantize.  The scratch comes from a fixed
     library-owned device array; ``out`` should then hold preallocated outputs.
     Calls that overlap on the GPU race on that shared scratch."""
-    _require_cuda(q, k)
+    with torch.cuda.device(_require_cuda(q, k)):
+        return _quant_qk_noalloc(q, k, tensor_layout, cu_seqlens, problem, out, granularity)
+
+
+def _quant_qk_noalloc(q, k, tensor_layout, cu_seqlens, problem, out, granularity):
     p = problem or Problem.from_tensors(q, k, tensor_layout, cu_seqlens, granularity)
     z = out or Quantized(p, tensor_layout)
     dev = q.device
@@ -185,19 +205,54 @@ def quant_qk_noalloc(q, k, tensor_layout="HND", cu_seqlens=None, problem=None,
 
 
 def quant_v(v, z: Quantized, workspace=None) -> Quantized:
-    """Per-channel e4m3 quantization of V, written token-contiguous (sage_quant_v)."""
-    _require_cuda(v)
-    p = z.problem
-    dev = v.device
-    if z.v8 is None:
-        z.v8 = torch.empty((p.heads_kv, p.head_dim, p.t_pad), dtype=torch.uint8, device=dev)
-        z.v_scale = torch.empty((p.batch, p.heads_kv, p.head_dim), dtype=torch.float32, device=dev)
-    ws = workspace if workspace is not None else _alloc(p.sizes.workspace_v, torch.float32, dev)
-    st = L.lib().sage_quant_v(ctypes.byref(p.c), _ptr(v), _strides(v, z.tensor_layout, p.varlen),
-                              _ptr(z.v8), _ptr(z.v_scale), _ptr(ws), ws.numel() * ws.element_size(),
-                              _stream())
-    L.check("sage_quant_v", st)
-    return z
+    """Per-channel e4m3 quantization of V, written token-contiguous (sage_quant_v).
+    With the 16-bit PV format V keeps its values, transposed the same way."""
+    with torch.cuda.device(_require_cuda(v)):
+        p = z.problem
+        dev = v.device
+        if z.v8 is None:
+            vt = torch.uint8 if p.pv == "fp8" else v.dtype
+            z.v8 = torch.empty((p.heads_kv, p.head_dim, p.t_pad), dtype=vt, device=dev)
+            z.v_scale = torch.empty((p.batch, p.heads_kv, p.head_dim), dtype=torch.float32, device=dev)
+        need = int(p.sizes.workspace_v)
+        ws = workspace if workspace is not None else (_alloc(need, torch.float32, dev) if need else None)
+        nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+        st = L.lib().sage_quant_v(ctypes.byref(p.c), _ptr(v), _strides(v, z.tensor_layout, p.varlen),
+                                  _ptr(z.v8), _ptr(z.v_scale), _ptr(ws), nbytes, _stream())
+        L.check("sage_quant_v", st)
+        return z
+
+
+def quant_qkv(q, k, v, tensor_layout="HND", cu_seqlens=None, problem=None, out: Quantized = None,
+              workspace=None, granularity="block", pv="fp8") -> Quantized:
+    """quant_qk and quant_v in one cooperative launch (sage_quant_qkv); the buffers are
+    bit-identical to the two separate calls."""
+    with torch.cuda.device(_require_cuda(q, k, v)):
+        p = problem or Problem.from_tensors(q, k, tensor_layout, cu_seqlens, granularity, pv)
+        z = out or Quantized(p, tensor_layout)
+        dev = q.device
+        d, tp = p.head_dim, p.t_pad
+        if z.q8 is None:
+            z.q8 = torch.empty((p.heads_q, tp, d), dtype=torch.int8, device=dev)
+            z.q_scale = torch.empty((p.heads_q, tp // p.q_block), dtype=torch.float32, device=dev)
+            z.k8 = torch.empty((p.heads_kv, tp, d), dtype=torch.int8, device=dev)
+            z.k_scale = torch.empty((p.heads_kv, tp // p.k_block), dtype=torch.float32, device=dev)
+            z.k_mean = torch.empty((p.batch, p.heads_kv, d), dtype=torch.float32, device=dev)
+        if z.v8 is None:
+            vt = torch.uint8 if p.pv == "fp8" else v.dtype
+            z.v8 = torch.empty((p.heads_kv, d, tp), dtype=vt, device=dev)
+            z.v_scale = torch.empty((p.batch, p.heads_kv, d), dtype=torch.float32, device=dev)
+        need = int(p.sizes.workspace_qkv)
+        ws = workspace if workspace is not None else _alloc(need + 256, torch.uint8, dev)
+        base = (ws.data_ptr() + 255) // 256 * 256
+        nbytes = ws.numel() * ws.element_size() - (base - ws.data_ptr())
+        st = L.lib().sage_quant_qkv(
+            ctypes.byref(p.c), _ptr(q), _strides(q, tensor_layout, p.varlen),
+            _ptr(k), _strides(k, tensor_layout, p.varlen), _ptr(v), _strides(v, tensor_layout, p.varlen),
+            _ptr(z.q8), _ptr(z.q_scale), _ptr(z.k8), _ptr(z.k_scale), _ptr(z.k_mean),
+            _ptr(z.v8), _ptr(z.v_scale), ctypes.c_void_p(base), nbytes, _stream())
+        L.check("sage_quant_qkv", st)
+        return z
 
 
 def _out_shape(p: Problem, layout: str):
@@ -211,6 +266,11 @@ def _out_shape(p: Problem, layout: str):
 def attn_fwd(z: Quantized, is_causal=False, sm_scale=None, out_dtype=None, out=None,
              return_lse=False):
     """The attention kernel on quantized operands (sage_attn_fwd)."""
+    with torch.cuda.device(_require_cuda(z.q8, z.k8, z.v8)):
+        return _attn_fwd(z, is_causal, sm_scale, out_dtype, out, return_lse)
+
+
+def _attn_fwd(z, is_causal, sm_scale, out_dtype, out, return_lse):
     p = z.problem
     dev = z.q8.device
     if out is None:
@@ -229,11 +289,12 @@ def attn_fwd(z: Quantized, is_causal=False, sm_scale=None, out_dtype=None, out=N
 
 
 def sageattn(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, cu_seqlens=None,
-             out_dtype=None, return_lse=False, granularity="block"):
-    """Quantized attention: smoothing + INT8 Q/K, FP8 V, then the fused attention kernel.
-    granularity="thread" selects a Q scale per token and a K scale per 32 tokens."""
-    z = quant_qk(q, k, tensor_layout, cu_seqlens, granularity=granularity)
-    quant_v(v, z)
+             out_dtype=None, return_lse=False, granularity="block", pv="fp8"):
+    """Quantized attention: smoothing + INT8 Q/K and FP8 V in one launch (quant_qkv),
+    then the fused attention kernel.
+    granularity="thread" selects a Q scale per token and a K scale per 32 tokens;
+    pv="fp16" runs P V in the input's 16-bit type instead of e4m3."""
+    z = quant_qkv(q, k, v, tensor_layout, cu_seqlens, granularity=granularity, pv=pv)
     return attn_fwd(z, is_causal=is_causal, sm_scale=sm_scale, out_dtype=out_dtype,
                     return_lse=return_lse)
 
@@ -243,7 +304,7 @@ _HOST_WS = {}
 
 def sageattn_host(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, out=None,
                   out_dtype=None, kv_heads_per_chunk=0, device=None, synchronize=True,
-                  granularity="block"):
+                  granularity="block", pv="fp8"):
     """sageattn on host tensors (sage_attn_host): chunks of heads are copied in,
     computed and copied out with the copies overlapping the kernels.
 
@@ -269,7 +330,7 @@ def sageattn_host(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, 
         code = 1
     else:
         raise ValueError(f"tensor_layout must be HND or NHD, got {tensor_layout}")
-    p = Problem(b, hq, hkv, n, d, q.dtype, granularity=granularity)
+    p = Problem(b, hq, hkv, n, d, q.dtype, granularity=granularity, pv=pv)
     odt = out_dtype or q.dtype
     if odt not in _OUT_DTYPES:
         raise TypeError(f"unsupported output dtype {odt}")
@@ -298,6 +359,11 @@ def sageattn_host(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, 
 
 def debug_qk_int32(z: Quantized, seq: int, head_q: int) -> torch.Tensor:
     """Exact int32 scores of one (sequence, query head) over its padded rows (test hook)."""
+    with torch.cuda.device(_require_cuda(z.q8, z.k8)):
+        return _debug_qk_int32(z, seq, head_q)
+
+
+def _debug_qk_int32(z, seq, head_q):
     p = z.problem
     n = (p.cu_list[seq + 1] - p.cu_list[seq]) if p.varlen else p.seqlen
     plen = -(-n // 128) * 128

@@ -1,7 +1,7 @@
 // attn_fwd.cuh - quantized attention forward on sm_100a tensor cores.
 //
 // Method (SageAttention): vibecrowd repo page "thu-ml--sageattention", How it
-// works (INT8 QK^T, FP8 PV, two-level accumulation for PV); heatdrop review
+// works (INT8 QK^T, FP8/FP16 PV, two-level accumulation for PV); heatdrop review
 // "2–5× attention speedups without the accuracy apology tour", The interesting
 // bit (two-level accumulation inside FP8 tensor cores) and Key highlights (GQA,
 // variable lengths); glossary page "SageAttention(セージアテンション)" (FlashAttention-
@@ -10,35 +10,42 @@
 // CTA = one (sequence, query head, 128-row Q tile).  16 warps in four warpgroups,
 // registers traded with setmaxnreg (128 x 40 + 128 x 88 + 256 x 192 = 512 x 128,
 // the launch allocation):
-//   WG0  warp 0: TMA producer (Q once, K / V tiles into 3-stage rings)
-//        warp 1: TMEM owner and MMA issuer (one thread); warps 2-3 idle
-//          S(j)  = Q8 K8(j)^T   tcgen05.mma kind::i8 -> TMEM buffer j % 2 (double-buffered)
-//          PV(j) = P8(j) V8(j)  tcgen05.mma kind::f8f6f4, A = P8 from TMEM -> fresh FP32
-//   WG1  softmax for keys 0-63 of every KV tile   (one thread per query row)
-//   WG2  softmax for keys 64-127 of every KV tile (one thread per query row)
+//   WG0  warp 0: TMA producer (Q once, K / V tiles into rings)
+//        warp 1: TMEM owner and S issuer, warp 2: PV issuer (one thread each); warp 3 idle
+//          S(j)  = Q8 K8(j)^T   tcgen05.mma kind::i8 -> TMEM S buffer j % 2
+//          PV(j) = P(j) V(j)    tcgen05.mma kind::f8f6f4 (e4m3) or kind::f16, A = P from
+//                               shared memory -> the PV block, a fresh FP32 accumulator
+//   WG1  softmax of the even KV tiles, WG2 of the odd ones (one thread per query row,
+//        a whole 128-key row each); consecutive tiles pass the running max through
+//        shared memory, so the two warpgroups work on different tiles at once
 //   WG3  two-level accumulation O = alpha O + PV(j) held in TMEM, and the epilogue
-// The two softmax warps of a lane quarter exchange their half-row maxima through
-// shared memory (one mbarrier per quarter and buffer), so both take the same running max.
 //
-// TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256,256+d) PV(j),
-// [384,384+d) running O.  In S buffer b, P8 of keys 0-63 goes to columns 0-15 and
-// of keys 64-127 to columns 64-79 (4 e4m3 per column), each over columns its own
-// softmax warps have already read; the PV MMA takes one TMEM address per 32-key step.
+// TMEM columns: S buffer 0 [0,128) (even tiles), S buffer 1 [128,256) (odd tiles),
+// the PV block [256, 256 + d) and the running O [384, 384 + d).  A softmax warpgroup
+// loads its S tile into registers and frees the buffer at once (P goes to shared
+// memory), so S(j + 2) can be computed while P(j) is being formed; the PV block and
+// the correction that folds it into O run behind, off the softmax's path.
 // Every S accumulates onto the magic pattern 0x4B400000 (fp32 1.5 * 2^23), so TMEM
 // returns bits(12582912 + S).  The pattern is written by the tensor core itself: before
 // the INT8 steps of S(j), one kind::f16 MMA with constant operands (every A entry 512,
 // every B entry 1536, K = 16, no accumulate) sets every element of the buffer to the
-// fp32 value 16 * 512 * 1536 = 12582912, and the INT8 steps add S onto those bits as
-// int32.  A buffer is free for S(j + 2) once the softmax warps have read S(j) and
-// written P8(j), and PV(j) has read P8(j).
+// fp32 value 16 * 512 * 1536 = 12582912, and the INT8 steps add S onto those bits.
 //
-// Per KV tile j, query row i (log2 domain, u = x * log2 e):
-//   u_j   = S_ij * (q_scale * k_scale_j * sm_scale * log2 e)
-//   m'    = max(m, max_j u_j);  alpha = 2^(m - m')
-//   p_j   = 2^(u_j - m' + log2 448)   (= 448 * exp(x_j - x_max'), exp2_poly below)
-//   l     = l * alpha + sum_j p_j     (unquantized), P8_j = e4m3(p_j) -> TMEM
-//   O     = O * alpha + PV_blk        (PV_blk = P8 V8 in FP32, fresh each tile)
-//   out   = O * v_scale / l ;  lse = m' ln 2 + ln(l / 448)
+// Per KV tile j, query row i, natural-log logits x_ij = ((S_ij q_scale_i) k_scale_j) sm_scale:
+//   m'    = max(m, max_j x_ij)                      (fp64, as the definition)
+//   p_j   = ps exp(x_j - m')                        (ps = 448 for e4m3 P, 1 for 16-bit P)
+//   l     = l exp(m - m') + sum_j p_j   (unquantized),  P_j = round(p_j) -> smem
+//   O     = O exp(m - m') + PV_blk      (PV_blk = P V in FP32, fresh each tile)
+//   out   = O v_scale / l ;  lse = m' + ln(l / ps)
+// p is computed in the log2 domain from fp32 operations relative to each 32-key chunk's
+// own largest score, t = fma(S - S_max_c, c_c, nb_c) with c_c = q_scale k_scale_c sm_scale
+// log2 e and nb_c = S_max_c c_c - m' log2 e + log2 ps formed in fp64 and rounded once,
+// and 2^t is the hardware exponential (ex2.approx, within 2 ulp).  That p is within
+// about 15 fp32 ulps of the exact value whatever the logits' magnitude.  An e4m3 code
+// is an integer decided by p, so for e4m3 P every p within 32 ulps of a rounding
+// midpoint is recomputed in fp64 from the definition and rounded from there: the codes
+// are those of the fp64 definition.  (A 16-bit P moves by one 16-bit ulp at such a
+// point; its codes are taken from the fast p.)
 #pragma once
 
 #include <type_traits>
@@ -56,47 +63,59 @@ constexpr int kSoftmaxRegs = 192;
 static_assert(128 * kProducerRegs + 128 * kCorrectionRegs + 256 * kSoftmaxRegs <=
                   kAttnThreads * kAttnLaunchRegs,
               "register split exceeds the launch allocation");
-constexpr int kKStages = 3;
-constexpr int kVStages = 3;
-constexpr float kLog2E = 1.4426950408889634f;
-constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
-constexpr float kLn448 = 6.104793232414985f;     // ln(448)
+constexpr double kLog2E64 = 1.4426950408889634;
+constexpr double kLog2_448_64 = 8.807354922057604;  // log2(448)
+constexpr float kLn448 = 6.104793232414985f;         // ln(448)
+constexpr int kAlphaRing = 4;                        // alpha slots between softmax and correction
+
+// PV operand formats: P and V in e4m3 (the method), or both in the input's 16-bit type
+enum : int { kPvE4m3 = 0, kPvF16 = 1, kPvBf16 = 2 };
 
 struct AttnArgs {
-  const float* q_scale;  // [Hq][T_pad/128]
-  const float* k_scale;  // [Hkv][T_pad/64]
-  const float* v_scale;  // [B][Hkv][D]
+  const float* q_scale;  // [Hq][T_pad/128], or [Hq][T_pad] with the per-thread granularity
+  const float* k_scale;  // [Hkv][T_pad/64], or [Hkv][T_pad/32]
+  const float* v_scale;  // [B][Hkv][D] (e4m3 PV only)
   void* out;
   int out_dtype;  // 0 fp16, 1 bf16, 2 fp32
   int64_t osb, osh, ost;
   float* lse;  // [Hq][T_pad] or null
   int hq, hkv, group;
-  float scale_log2;  // sm_scale * log2(e)
+  double scale;  // sm_scale (1/sqrt(d) by default), fp64 as in the definition
   int causal;
-  int fine;  // per-thread granularity: q_scale per token, k_scale per 32-token block
 };
 
-template <int D>
-struct AttnSmem {
-  static constexpr int kTileQ = kBlkQ * D;    // bytes of one Q (or K) tile
-  static constexpr int kTileV = D * kKvTile;  // bytes of one V^T tile
+template <int D, int PV>
+struct AttnCfg {
+  static constexpr int kEB = PV == kPvE4m3 ? 1 : 2;      // bytes per P / V element
+  static constexpr int kKS = PV == kPvE4m3 ? 3 : 2;      // K ring stages
+  static constexpr int kVS = PV == kPvE4m3 ? 3 : 2;      // V ring stages
+  static constexpr int kPBufs = PV == kPvE4m3 ? 3 : 2;   // P tiles in shared memory
+  static constexpr int kTileQK = kBlkQ * D;              // bytes of one Q (or K) tile
+  static constexpr int kTileV = D * kKvTile * kEB;       // bytes of one V^T tile
+  static constexpr int kTileP = kBlkQ * kKvTile * kEB;   // bytes of one P tile
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kTileQ;
-  static constexpr int kVOff = kKOff + kKStages * kTileQ;
-  static constexpr int kXOff = kVOff + kVStages * kTileV;  // float xchg[2][2][128]
-  static constexpr int kAOff = kXOff + 2 * 2 * 128 * 4;    // float alpha[2][128]
-  static constexpr int kLOff = kAOff + 2 * 128 * 4;        // float lfin[2][128], mfin[128]
+  static constexpr int kKOff = kQOff + kTileQK;
+  static constexpr int kVOff = kKOff + kKS * kTileQK;
+  static constexpr int kPOff = kVOff + kVS * kTileV;
   // constant f16 operands of the prefill MMA: 128 rows x 128 B each (128-byte swizzle
   // atoms; every entry equal, so the layout is immaterial)
-  static constexpr int kCAOff = ((kLOff + 3 * 128 * 4) + 1023) / 1024 * 1024;
+  static constexpr int kCAOff = kPOff + kPBufs * kTileP;
   static constexpr int kCBOff = kCAOff + 128 * 128;
-  static constexpr int kBarOff = kCBOff + 128 * 128;
-  // barriers: q_full, k_full[3], k_empty[3], v_full[3], v_empty[3], s_full[2], s_free[2],
-  // p_full[2], pv_full, pv_free, epi, mma_done, xchg[2][4] -> 31
-  static constexpr int kNumBars = 31;
+  static constexpr int kMOff = kCBOff + 128 * 128;              // double mrun[2][128]
+  static constexpr int kAOff = kMOff + 2 * 128 * 8;             // float alpha[4][128]
+  static constexpr int kLOff = kAOff + kAlphaRing * 128 * 4;    // float lfin[2][128]
+  static constexpr int kFOff = kLOff + 2 * 128 * 4;             // double mfin[2][128]
+  static constexpr int kBarOff = kFOff + 2 * 128 * 8;
+  // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS],
+  // s_full[2], s_free[2], m_ready[2], p_full[PB], p_free[PB], a_full[4], a_free[4],
+  // pv_full, pv_free, epi, done
+  static constexpr int kBarK = 1, kBarV = kBarK + 2 * kKS, kBarS = kBarV + 2 * kVS;
+  static constexpr int kBarP = kBarS + 6, kBarA = kBarP + 2 * kPBufs, kBarX = kBarA + 2 * kAlphaRing;
+  static constexpr int kNumBars = kBarX + 4;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kSlotOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
+  static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -105,32 +124,9 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^t in plain IEEE fp32 operations, so that the P8 code it decides can be
-// reproduced exactly on any host: Cody-Waite split t = n + f with n = rint(t)
-// taken by magic-number rounding (r = t + 1.5 * 2^23, bits(r) = 0x4B400000 + n)
-// and f = t - (r - 1.5 * 2^23) in [-1/2, 1/2], a degree-2 polynomial for 2^f
-// (coefficients fitted for minimal relative error with the constant term fixed at
-// 1, so integer t gives exact powers of two; max relative error 1.97e-3, well below
-// the e4m3 step of P, which is 6.25% to 12.5%), and n added to the exponent field,
-// clamped below at -125 so the result stays a normal number.
-constexpr float kExp2C1 = 0.702944696f;  // 0x3f33f42f
-constexpr float kExp2C2 = 0.239866376f;  // 0x3e759f88
-constexpr int kExpClampBits = 0x4B400000 - 125;
-__device__ __forceinline__ float exp2_poly(float t) {
-  const float r = __fadd_rn(t, 12582912.0f);
-  const float f = __fsub_rn(t, __fsub_rn(r, 12582912.0f));
-  float p = __fmaf_rn(kExp2C2, f, kExp2C1);
-  p = __fmaf_rn(p, f, 1.0f);
-  const int rb = max(__float_as_int(r), kExpClampBits);
-  return __int_as_float(__float_as_int(p) + rb * (1 << 23));
-}
-
-// ---- packed fp32 pair arithmetic (one instruction per two values); element 0 of a
-// pair is .x, handed to the f32x2 instructions as the low half of a 64-bit register.
+// ---- packed fp32 pair arithmetic (one instruction per two values)
 using f2 = float2;
 __device__ __forceinline__ f2 f2_make(float lo, float hi) { return make_float2(lo, hi); }
-__device__ __forceinline__ float f2_lo(f2 a) { return a.x; }
-__device__ __forceinline__ float f2_hi(f2 a) { return a.y; }
 __device__ __forceinline__ f2 f2_fma(f2 a, f2 b, f2 c) {
   f2 d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(reinterpret_cast<uint64_t&>(d)) : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)), "l"(reinterpret_cast<const uint64_t&>(c)));
@@ -160,8 +156,8 @@ __device__ __forceinline__ void tmem_wait_ld_tied(uint32_t (&r)[32]) {
                :
                : "memory");
 }
-__device__ __forceinline__ void tmem_wait_ld_tied(uint32_t (&a)[32], uint32_t (&b)[32]) {
-  tmem_wait_ld_tied(a);
+// Registers already covered by a preceding wait: only pins them after it.
+__device__ __forceinline__ void pin_regs(uint32_t (&b)[32]) {
   asm volatile(""
                : "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]),
                  "+r"(b[6]), "+r"(b[7]), "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]),
@@ -175,16 +171,16 @@ __device__ __forceinline__ void tmem_wait_ld_tied(uint32_t (&a)[32], uint32_t (&
 __device__ __forceinline__ f2 pair_of(const uint32_t (&r)[32], int k) {
   return f2_make(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
 }
-// The S region is pre-filled with kMagicBits (the fp32 1.5 * 2^23 = 12582912) and the
+// The S buffer is pre-filled with kMagicBits (the fp32 1.5 * 2^23 = 12582912) and the
 // INT8 MMAs accumulate onto it, so TMEM returns bits(12582912 + S): an fp32 whose
 // value is exactly 12582912 + S for |S| < 2^22 (|S| <= d * 127^2 here).  Those values
-// are positive and ordered like S, and S itself is one exact subtraction away.
+// are positive and ordered like S, and any difference of two is exact.
 constexpr uint32_t kMagicBits = 0x4B400000u;
 constexpr float kMagic = 12582912.0f;
 
-// max of acc and 32 magic-offset scores (masked entries hold 0, below every valid value)
-__device__ __forceinline__ float max32(const uint32_t (&r)[32], float acc) {
-  float m0 = acc, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
+// max of 32 magic-offset scores (masked entries hold 0, below every valid value)
+__device__ __forceinline__ float max32(const uint32_t (&r)[32]) {
+  float m0 = 0.0f, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
 #pragma unroll
   for (int i = 0; i < 32; i += 8) {
     m0 = fmax3(m0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
@@ -195,80 +191,183 @@ __device__ __forceinline__ float max32(const uint32_t (&r)[32], float acc) {
   return fmax3(m0, m1, fmaxf(m2, m3));
 }
 
-// P for 32 keys of one 64-key half: S = (12582912 + S) - 12582912 (exact),
-// t = fma(S, ck, log2 448 - m'), p = exp2_poly(t) evaluated two values per
-// instruction (the same fp32 operations as exp2_poly).  Returns the e4m3 codes
-// packed four per word and adds p into acc.  With kMasked, key i is kept only
-// when bit i of `keep` is set; dropped keys get p = 0.
-template <bool kMasked>
-__device__ __forceinline__ void p8_chunk(const uint32_t (&r)[32], float ck, float nb, f2& acc,
-                                         uint32_t (&w)[8], uint32_t keep) {
-  const f2 CK = f2_make(ck, ck), NB = f2_make(nb, nb);
-  const f2 M = f2_make(kMagic, kMagic), NM = f2_make(-kMagic, -kMagic);
-  const f2 NEG1 = f2_make(-1.0f, -1.0f), ONE = f2_make(1.0f, 1.0f);
-  const f2 C1 = f2_make(kExp2C1, kExp2C1), C2 = f2_make(kExp2C2, kExp2C2);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    f2 pp[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const f2 t = f2_fma(f2_add(pair_of(r, 2 * i + h), NM), CK, NB);
-      const f2 rr = f2_add(t, M);
-      const f2 f = f2_fma(f2_add(rr, NM), NEG1, t);
-      f2 p = f2_fma(C2, f, C1);
-      p = f2_fma(p, f, ONE);
-      // bits(rr) = 0x4B400000 + n: max() clamps n at -125, and bits << 23 is n << 23
-      // modulo 2^32
-      uint32_t lo = __float_as_uint(p.x) + (static_cast<uint32_t>(max(__float_as_int(rr.x), kExpClampBits)) << 23);
-      uint32_t hi = __float_as_uint(p.y) + (static_cast<uint32_t>(max(__float_as_int(rr.y), kExpClampBits)) << 23);
-      if (kMasked) {
-        const int e = 4 * i + 2 * h;
-        lo = ((keep >> e) & 1u) ? lo : 0u;
-        hi = ((keep >> (e + 1)) & 1u) ? hi : 0u;
-      }
-      pp[h] = f2_make(__uint_as_float(lo), __uint_as_float(hi));
-    }
-    acc = f2_add(acc, f2_add(pp[0], pp[1]));
-    w[i] = e4m3x2(f2_lo(pp[0]), f2_hi(pp[0])) | (e4m3x2(f2_lo(pp[1]), f2_hi(pp[1])) << 16);
+// Two fp32 values -> the PV operand format, packed into 16 bits (`lo` in the low half).
+template <int PV>
+__device__ __forceinline__ uint32_t cvt_pair(float lo, float hi) {
+  if constexpr (PV == kPvE4m3) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+  } else if constexpr (PV == kPvF16) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+  } else {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
   }
 }
 
-template <int D, class Seq>
+// ---- exact e4m3 decision near a rounding midpoint
+// In the e4m3 normal range (p >= 2^-6) a code boundary is a value whose fp32 bits have
+// their low 20 bits equal to 0x80000 (the fp32 mantissa's first three bits are kept).
+// A fast p within kMidWin ulps of such a boundary is flagged: c = bits(p) + kMidWin has
+// (c & kMidMask) == 0x80000 exactly then.
+constexpr uint32_t kMidWin = 32;
+constexpr uint32_t kMidMask = 0xFFFFFu & ~(2u * kMidWin - 1u);
+__device__ __forceinline__ uint32_t mid_flag(float p) {  // 0 iff p is flagged
+  return ((__float_as_uint(p) + kMidWin) & kMidMask) ^ 0x80000u;
+}
+
+// The value to convert for a flagged element: the definition's p64 = 448 exp(x - m) with
+// x = ((S q_scale) k_scale) sm_scale in fp64, placed on the right side of the midpoint
+// next to the fast p (one fp32 ulp away, or the midpoint itself for an exact tie, which
+// the conversion then rounds to even, as the definition does).  Below the e4m3 normal
+// range, or at the saturation end, the fast p is kept.
+__device__ __noinline__ float p_at_midpoint(float s, float sq, float sk, double scale, double m64,
+                                            float p_fast) {
+  const uint32_t mid_bits = ((__float_as_uint(p_fast) + kMidWin) & 0xFFF00000u) | 0x80000u;
+  const float mid = __uint_as_float(mid_bits);
+  if (!(mid >= 0x1p-6f) || mid > 448.0f) return p_fast;
+  const double x = ((static_cast<double>(s) * static_cast<double>(sq)) * static_cast<double>(sk)) * scale;
+  const double p = 448.0 * exp(x - m64);
+  const double md = static_cast<double>(mid);
+  if (p > md) return __uint_as_float(mid_bits + 1u);
+  if (p < md) return __uint_as_float(mid_bits - 1u);
+  return mid;
+}
+
+// P for the 32 keys of chunk c of one row: t = fma(S - S_max_c, ck, nb) (the difference
+// of two magic-offset floats is exact), p = 2^t, added into acc and written, in the PV
+// operand format, to the row's slot of a 128-byte-swizzled K-major P tile in shared
+// memory (`prow` = tile base + row * 128, `rx` = row % 8).  With kMasked, key i is kept
+// only when bit i of `keep` is set; dropped keys get p = 0.  With kExact (e4m3 P) codes
+// of p near a rounding midpoint are decided in fp64 by p_at_midpoint.
+struct ChunkExact {
+  float sq, sk;
+  double scale, m64;
+};
+
+// The 32 e4m3 codes of a chunk again, with every flagged p decided from the definition.
+// Rare (a flag hits about 6e-5 of the elements), so kept out of line: the chunk's scores
+// come in through local memory and the eight code words go back the same way.  The
+// fast p is recomputed with the same fp32 operations, so unflagged codes are unchanged.
+__device__ __noinline__ void e4m3_codes_exact(const uint32_t* s32, float hmax, float ck, float nb,
+                                             uint32_t keep, ChunkExact ex, uint32_t* w) {
+#pragma unroll 1
+  for (int i = 0; i < 32; i += 2) {
+    float p[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float sv = __uint_as_float(s32[i + e]);
+      p[e] = ((keep >> (i + e)) & 1u) ? ex2(__fmaf_rn(__fsub_rn(sv, hmax), ck, nb)) : 0.0f;
+      if (mid_flag(p[e]) == 0u) p[e] = p_at_midpoint(sv - kMagic, ex.sq, ex.sk, ex.scale, ex.m64, p[e]);
+    }
+    uint16_t two;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(two) : "f"(p[1]), "f"(p[0]));
+    if ((i >> 1) & 1) w[i >> 2] |= static_cast<uint32_t>(two) << 16;
+    else w[i >> 2] = two;
+  }
+}
+
+template <int PV, bool kMasked, bool kExact>
+__device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], float hmax, float ck, float nb,
+                                        f2& acc, uint32_t keep, uint32_t prow, int rx, int c,
+                                        const ChunkExact& ex) {
+  const f2 CK = f2_make(ck, ck), NB = f2_make(nb, nb), NH = f2_make(-hmax, -hmax);
+  // one 16-byte chunk of the row at a time: 16 e4m3 codes or 8 16-bit values
+  constexpr int kPerChunk = PV == kPvE4m3 ? 16 : 8;
+  constexpr int kStores = 32 / kPerChunk;
+  uint32_t w[kStores * 4];
+  uint32_t zmin = 0xFFFFFFFFu;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const f2 t = f2_fma(f2_add(pair_of(r, i), NH), CK, NB);
+    float p0 = ex2(t.x), p1 = ex2(t.y);
+    if (kMasked) {
+      p0 = ((keep >> (2 * i)) & 1u) ? p0 : 0.0f;
+      p1 = ((keep >> (2 * i + 1)) & 1u) ? p1 : 0.0f;
+    }
+    acc = f2_add(acc, f2_make(p0, p1));
+    if constexpr (kExact) zmin = min(zmin, min(mid_flag(p0), mid_flag(p1)));
+    const uint32_t two = cvt_pair<PV>(p0, p1);
+    if constexpr (PV == kPvE4m3) {
+      if (i & 1) w[i >> 1] |= two << 16; else w[i >> 1] = two;
+    } else {
+      w[i] = two;
+    }
+  }
+  if constexpr (kExact) {
+    if (__any_sync(0xffffffffu, zmin == 0u) && zmin == 0u) {
+      uint32_t s32[32], wx[8];  // local copies: w itself stays in registers
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s32[i] = r[i];
+      e4m3_codes_exact(s32, hmax, ck, nb, kMasked ? keep : 0xFFFFFFFFu, ex, wx);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = wx[i];
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < kStores; ++e) {
+    if constexpr (PV == kPvE4m3) {
+      // 32 codes = 16-byte chunks 2c, 2c + 1 of the 128-byte row
+      st_shared16(prow + ((((2 * c + e) ^ rx) & 7) << 4), w[4 * e], w[4 * e + 1], w[4 * e + 2],
+                  w[4 * e + 3]);
+    } else {
+      // 64 bytes = 16-byte chunks 4c .. 4c + 3 of the 256-byte row; keys 0-63 fill
+      // swizzle block 0 and keys 64-127 block 1 (128 rows x 128 B each)
+      const int g = 4 * c + e;
+      st_shared16(prow + ((g >> 3) * (kBlkQ * 128)) + ((((g & 7) ^ rx) & 7) << 4), w[4 * e],
+                  w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+    }
+  }
+}
+
+template <int D, class Seq, bool kFine, int PV>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v,
                      const __grid_constant__ Seq seq, const __grid_constant__ AttnArgs a) {
-  using L = AttnSmem<D>;
+  using L = AttnCfg<D, PV>;
+  constexpr int KS = L::kKS, VS = L::kVS, PB = L::kPBufs;
+  constexpr bool kExact = PV == kPvE4m3;
   constexpr uint32_t kSwizzle = (D == 128) ? 2u : 4u;  // UMMA layout type: 128B / 64B swizzle
   constexpr uint32_t kSboQK = 8u * D;                  // 8 rows of D bytes
   constexpr uint32_t kIdescS = idesc_i8(128, kKvTile);
-  constexpr uint32_t kIdescPV = idesc_e4m3_f32(128, D);
+  constexpr uint32_t kIdescPV = PV == kPvE4m3 ? idesc_e4m3_f32(128, D)
+                                : PV == kPvF16 ? idesc_f16_f32(128, D) : idesc_bf16_f32(128, D);
   constexpr uint32_t kIdescPre = idesc_f16_f32(128, kKvTile);
   constexpr uint32_t kColPV = 256, kColO = 384;
+  constexpr double kLog2Ps = PV == kPvE4m3 ? kLog2_448_64 : 0.0;
+  constexpr float kLnPs = PV == kPvE4m3 ? kLn448 : 0.0f;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + L::kBarOff;
-  auto bar_q = [&]() { return bar0; };
-  auto bar_kf = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto bar_ke = [&](int s) { return bar0 + 8u * (4 + s); };
-  auto bar_vf = [&](int s) { return bar0 + 8u * (7 + s); };
-  auto bar_ve = [&](int s) { return bar0 + 8u * (10 + s); };
-  auto bar_sfull = [&](int b) { return bar0 + 8u * (13 + b); };
-  auto bar_sfree = [&](int b) { return bar0 + 8u * (15 + b); };
-  auto bar_pfull = [&](int b) { return bar0 + 8u * (17 + b); };
-  const uint32_t bar_pvfull = bar0 + 8u * 19;
-  const uint32_t bar_pvfree = bar0 + 8u * 20;
-  const uint32_t bar_epi = bar0 + 8u * 21;
-  const uint32_t bar_done = bar0 + 8u * 22;
-  // the two softmax warps of lane quarter q swap half-row maxima through xchg
-  auto bar_xchg = [&](int buf, int q) { return bar0 + 8u * (23 + 4 * buf + q); };
-  float* xchg = reinterpret_cast<float*>(smem + L::kXOff);  // [buffer][half][row]
-  float* alph = reinterpret_cast<float*>(smem + L::kAOff);  // [buffer][row]
-  float* lfin = reinterpret_cast<float*>(smem + L::kLOff);  // [half][row], then mfin[row]
+  const uint32_t bar_q = bar0;
+  auto bar_kf = [&](int s) { return bar0 + 8u * (L::kBarK + s); };
+  auto bar_ke = [&](int s) { return bar0 + 8u * (L::kBarK + KS + s); };
+  auto bar_vf = [&](int s) { return bar0 + 8u * (L::kBarV + s); };
+  auto bar_ve = [&](int s) { return bar0 + 8u * (L::kBarV + VS + s); };
+  auto bar_sfull = [&](int b) { return bar0 + 8u * (L::kBarS + b); };
+  auto bar_sfree = [&](int b) { return bar0 + 8u * (L::kBarS + 2 + b); };
+  auto bar_mready = [&](int b) { return bar0 + 8u * (L::kBarS + 4 + b); };
+  auto bar_pfull = [&](int b) { return bar0 + 8u * (L::kBarP + b); };
+  auto bar_pfree = [&](int b) { return bar0 + 8u * (L::kBarP + PB + b); };
+  auto bar_afull = [&](int b) { return bar0 + 8u * (L::kBarA + b); };
+  auto bar_afree = [&](int b) { return bar0 + 8u * (L::kBarA + kAlphaRing + b); };
+  const uint32_t bar_pvfull = bar0 + 8u * L::kBarX;
+  const uint32_t bar_pvfree = bar_pvfull + 8u;
+  const uint32_t bar_epi = bar_pvfull + 16u;
+  const uint32_t bar_done = bar_pvfull + 24u;
+  double* mrun = reinterpret_cast<double*>(smem + L::kMOff);   // [tile % 2][row], fp64 max
+  float* alph = reinterpret_cast<float*>(smem + L::kAOff);     // [tile % 4][row]
+  float* lfin = reinterpret_cast<float*>(smem + L::kLOff);     // [wg][row]
+  double* mfin = reinterpret_cast<double*>(smem + L::kFOff);   // [wg][row]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -307,19 +406,26 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
-    mbar_init(bar_q(), 1);
-    for (int s = 0; s < kKStages; ++s) { mbar_init(bar_kf(s), 1); mbar_init(bar_ke(s), 1); }
-    for (int s = 0; s < kVStages; ++s) { mbar_init(bar_vf(s), 1); mbar_init(bar_ve(s), 1); }
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < KS; ++s) { mbar_init(bar_kf(s), 1); mbar_init(bar_ke(s), 1); }
+    for (int s = 0; s < VS; ++s) { mbar_init(bar_vf(s), 1); mbar_init(bar_ve(s), 1); }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar_sfull(s), 1);
-      mbar_init(bar_sfree(s), 12);  // 8 softmax warps + 4 correction warps re-arm buffer s
-      mbar_init(bar_pfull(s), 8);   // 8 softmax warps wrote P (and alpha) into buffer s
+      mbar_init(bar_sfull(s), 1);   // tcgen05.commit of S
+      mbar_init(bar_sfree(s), 4);   // the 4 softmax warps of the tile loaded S
+      mbar_init(bar_mready(s), 4);  // the 4 softmax warps of the tile published its max
     }
-    mbar_init(bar_pvfull, 1);
-    mbar_init(bar_pvfree, 4);
+    for (int s = 0; s < PB; ++s) {
+      mbar_init(bar_pfull(s), 4);   // the 4 softmax warps wrote P
+      mbar_init(bar_pfree(s), 1);   // tcgen05.commit of the PV that read it
+    }
+    for (int s = 0; s < kAlphaRing; ++s) {
+      mbar_init(bar_afull(s), 4);   // the 4 softmax warps wrote the tile's alpha
+      mbar_init(bar_afree(s), 4);   // the 4 correction warps read it
+    }
+    mbar_init(bar_pvfull, 1);       // tcgen05.commit of PV
+    mbar_init(bar_pvfree, 4);       // the 4 correction warps read the PV block
     mbar_init(bar_epi, 8);
-    mbar_init(bar_done, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(bar_xchg(i >> 2, i & 3), 2);
+    mbar_init(bar_done, 2);         // a commit from each MMA issuer
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -352,183 +458,227 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     if (warp == 0 && lane == 0 && !dead) {
       // ========================================================== TMA producer
       bool ok = true;
-      mbar_arrive_expect_tx(bar_q(), L::kTileQ);
-      tma_load_2d(sbase + L::kQOff, &tmap_q, 0, hq * seq.t_pad + off + qt * kBlkQ, bar_q());
+      mbar_arrive_expect_tx(bar_q, L::kTileQK);
+      tma_load_2d(sbase + L::kQOff, &tmap_q, 0, hq * seq.t_pad + off + qt * kBlkQ, bar_q);
       int nk = 0, nv = 0;  // loads issued
       for (int j = 0; j < nkv && ok; ++j) {
-        const int ks = j % kKStages, vs = j % kVStages;
-        if (j >= kKStages) ok = mbar_wait<true>(bar_ke(ks), ((j / kKStages) - 1) & 1, 0x101);
+        const int ks = j % KS, vs = j % VS;
+        if (j >= KS) ok = mbar_wait<true>(bar_ke(ks), ((j / KS) - 1) & 1, 0x101);
         if (!ok) break;
-        mbar_arrive_expect_tx(bar_kf(ks), L::kTileQ);
-        tma_load_2d(sbase + L::kKOff + ks * L::kTileQ, &tmap_k, 0,
+        mbar_arrive_expect_tx(bar_kf(ks), L::kTileQK);
+        tma_load_2d(sbase + L::kKOff + ks * L::kTileQK, &tmap_k, 0,
                     hk * seq.t_pad + off + j * kKvTile, bar_kf(ks));
         ++nk;
-        if (j >= kVStages) ok = mbar_wait<true>(bar_ve(vs), ((j / kVStages) - 1) & 1, 0x102);
+        if (j >= VS) ok = mbar_wait<true>(bar_ve(vs), ((j / VS) - 1) & 1, 0x102);
         if (!ok) break;
         mbar_arrive_expect_tx(bar_vf(vs), L::kTileV);
-        tma_load_2d(sbase + L::kVOff + vs * L::kTileV, &tmap_v, off + j * kKvTile, hk * D,
-                    bar_vf(vs));
+        if constexpr (PV == kPvE4m3) {
+          tma_load_2d(sbase + L::kVOff + vs * L::kTileV, &tmap_v, off + j * kKvTile, hk * D,
+                      bar_vf(vs));
+        } else {
+          // 16-bit V^T rows are 256 B per tile: two 128-byte-swizzled boxes of 64 keys
+          const int x = 2 * (off + j * kKvTile);
+          tma_load_2d(sbase + L::kVOff + vs * L::kTileV, &tmap_v, x, hk * D, bar_vf(vs));
+          tma_load_2d(sbase + L::kVOff + vs * L::kTileV + D * 128, &tmap_v, x + 128, hk * D,
+                      bar_vf(vs));
+        }
         ++nv;
       }
       // drain: the most recent load of every stage has landed before the CTA can exit
       const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait_sleep(bar_q(), 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
-      for (int jj = max(0, nk - kKStages); jj < nk; ++jj)
-        while (!mbar_try_wait_sleep(bar_kf(jj % kKStages), (jj / kKStages) & 1) &&
+      while (!mbar_try_wait_sleep(bar_q, 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
+      for (int jj = max(0, nk - KS); jj < nk; ++jj)
+        while (!mbar_try_wait_sleep(bar_kf(jj % KS), (jj / KS) & 1) &&
                global_timer_ns() - t0 < kWaitLimitNs) {}
-      for (int jj = max(0, nv - kVStages); jj < nv; ++jj)
-        while (!mbar_try_wait_sleep(bar_vf(jj % kVStages), (jj / kVStages) & 1) &&
+      for (int jj = max(0, nv - VS); jj < nv; ++jj)
+        while (!mbar_try_wait_sleep(bar_vf(jj % VS), (jj / VS) & 1) &&
                global_timer_ns() - t0 < kWaitLimitNs) {}
-    } else if (warp == 1 && lane == 0 && !dead) {
-      // ========================================================== MMA issuer
+    } else if ((warp == 1 || warp == 2) && lane == 0 && !dead) {
+      // ========================================================== MMA issuers
+      // warp 1 issues every S(j), warp 2 every PV(j); each waits (suspended) only on its
+      // own inputs.  A thread's tcgen05.mma ops run in its issue order and its commits
+      // track its own ops, and the two streams share no operand: S(j) writes S buffer
+      // j % 2 from Q and K(j), PV(j) writes the PV block from P(j) and V(j).
       // descriptors differ only in their start-address field (bits 0-13, address >> 4)
-      const uint64_t dq = sdesc_kmajor(sbase + L::kQOff, kSboQK, kSwizzle);
-      const uint64_t dk = sdesc_kmajor(sbase + L::kKOff, kSboQK, kSwizzle);
-      const uint64_t dv = sdesc_kmajor(sbase + L::kVOff, 1024u, 2u);
-      const uint64_t dca = sdesc_kmajor(sbase + L::kCAOff, 1024u, 2u);
-      const uint64_t dcb = sdesc_kmajor(sbase + L::kCBOff, 1024u, 2u);
-      auto issue_s = [&](int js) {  // S(js) = Q8 K8(js)^T onto the armed buffer js % 2
-        const int ks = js % kKStages;
-        const uint64_t bk = dk + static_cast<uint64_t>((ks * L::kTileQ) >> 4);
-        const uint32_t d_tmem = tmem + 128u * (js & 1);
-        mma_f16_ss(d_tmem, dca, dcb, kIdescPre, 0u);  // every element := 12582912.0f
-#pragma unroll
-        for (int s = 0; s < D / 32; ++s) mma_i8_ss(d_tmem, dq + 2u * s, bk + 2u * s, kIdescS, 1u);
-        tc_commit(bar_sfull(js & 1));
-        tc_commit(bar_ke(ks));
-      };
-      auto issue_pv = [&](int j) {  // PV(j) = P8(j) V8(j) into a fresh FP32 accumulator
-        const int vs = j % kVStages;
-        const uint64_t bv = dv + static_cast<uint64_t>((vs * L::kTileV) >> 4);
-        const uint32_t p_tmem = tmem + 128u * (j & 1);
-#pragma unroll
-        for (int s = 0; s < kKvTile / 32; ++s) {
-          // keys 32s..32s+31: P8 columns 0, 8 (first half) and 64, 72 (second half)
-          const uint32_t a_col = (s < 2) ? 8u * s : 64u + 8u * (s - 2);
-          mma_f8_ts(tmem + kColPV, p_tmem + a_col, bv + 2u * s, kIdescPV, s > 0 ? 1u : 0u);
-        }
-        tc_commit(bar_pvfull);
-        tc_commit(bar_ve(vs));
-      };
-      bool ok = mbar_wait<true>(bar_q(), 0, 0x201);
-      for (int js = 0; js < 2 && js < nkv && ok; ++js) {
-        ok = mbar_wait<true>(bar_kf(js % kKStages), (js / kKStages) & 1, 0x202) &&
-             mbar_wait<true>(bar_sfree(js & 1), 0, 0x203);
-        if (!ok) break;
-        tc_fence_after();
-        issue_s(js);
-      }
-      for (int j = 0; j < nkv && ok; ++j) {
-        ok = mbar_wait<true>(bar_pfull(j & 1), (j >> 1) & 1, 0x204) &&
-             mbar_wait<true>(bar_vf(j % kVStages), (j / kVStages) & 1, 0x205) &&
-             (j == 0 || mbar_wait<true>(bar_pvfree, (j - 1) & 1, 0x206));
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(j);
-        const int js = j + 2;
-        if (js < nkv) {
-          ok = mbar_wait<true>(bar_kf(js % kKStages), (js / kKStages) & 1, 0x207) &&
-               mbar_wait<true>(bar_sfree(js & 1), (js >> 1) & 1, 0x208);
+      bool ok = mbar_wait<true>(bar_q, 0, 0x201);
+      if (warp == 1) {
+        const uint64_t dq = sdesc_kmajor(sbase + L::kQOff, kSboQK, kSwizzle);
+        const uint64_t dk = sdesc_kmajor(sbase + L::kKOff, kSboQK, kSwizzle);
+        const uint64_t dca = sdesc_kmajor(sbase + L::kCAOff, 1024u, 2u);
+        const uint64_t dcb = sdesc_kmajor(sbase + L::kCBOff, 1024u, 2u);
+        for (int js = 0; js < nkv && ok; ++js) {
+          // S(js) needs K(js) and its buffer free (tile js - 2 loaded by its softmax)
+          ok = (js < 2 || mbar_wait(bar_sfree(js & 1), ((js >> 1) - 1) & 1, 0x202)) &&
+               mbar_wait(bar_kf(js % KS), (js / KS) & 1, 0x203);
           if (!ok) break;
           tc_fence_after();
-          issue_s(js);
+          const int ks = js % KS;
+          const uint64_t bk = dk + static_cast<uint64_t>((ks * L::kTileQK) >> 4);
+          const uint32_t d_tmem = tmem + 128u * (js & 1);
+          mma_f16_ss(d_tmem, dca, dcb, kIdescPre, 0u);  // every element := 12582912.0f
+#pragma unroll
+          for (int s = 0; s < D / 32; ++s) mma_i8_ss(d_tmem, dq + 2u * s, bk + 2u * s, kIdescS, 1u);
+          tc_commit(bar_sfull(js & 1));
+          tc_commit(bar_ke(ks));
+        }
+      } else {
+        const uint64_t dv = sdesc_kmajor(sbase + L::kVOff, 1024u, 2u);
+        const uint64_t dp = sdesc_kmajor(sbase + L::kPOff, 1024u, 2u);
+        for (int jp = 0; jp < nkv && ok; ++jp) {
+          // PV(jp) needs P(jp), V(jp) and the PV block free (tile jp - 1 read by the
+          // correction)
+          ok = mbar_wait(bar_pfull(jp % PB), (jp / PB) & 1, 0x204) &&
+               mbar_wait(bar_vf(jp % VS), (jp / VS) & 1, 0x205) &&
+               (jp == 0 || mbar_wait(bar_pvfree, (jp - 1) & 1, 0x206));
+          if (!ok) break;
+          tc_fence_after();
+          const int vs = jp % VS;
+          const uint64_t bv = dv + static_cast<uint64_t>((vs * L::kTileV) >> 4);
+          const uint64_t ap = dp + static_cast<uint64_t>(((jp % PB) * L::kTileP) >> 4);
+          const uint32_t d_tmem = tmem + kColPV;
+          if constexpr (PV == kPvE4m3) {
+#pragma unroll
+            for (int s = 0; s < kKvTile / 32; ++s)  // 32 keys (32 bytes) per step
+              mma_f8_ss(d_tmem, ap + 2u * s, bv + 2u * s, kIdescPV, s > 0 ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int s = 0; s < kKvTile / 16; ++s) {  // 16 keys (32 bytes) per step
+              const uint32_t blk = s >> 2, w = s & 3;  // 64-key swizzle block, step within it
+              mma_f16_ss(d_tmem, ap + ((blk * (kBlkQ * 128) + w * 32) >> 4),
+                         bv + ((blk * (D * 128) + w * 32) >> 4), kIdescPV, s > 0 ? 1u : 0u);
+            }
+          }
+          tc_commit(bar_pvfull);
+          tc_commit(bar_ve(vs));
+          tc_commit(bar_pfree(jp % PB));
         }
       }
       // every MMA issued by this thread has completed before TMEM is released
       tc_commit(bar_done);
-      const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait_sleep(bar_done, 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
+      const uint64_t t1 = global_timer_ns();
+      while (!mbar_try_wait_sleep(bar_done, 0) && global_timer_ns() - t1 < kWaitLimitNs) {}
     }
   } else if (wg <= 2) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-    // ============================================================ softmax (one 64-key half)
-    const int h = wg - 1;           // 0: keys 0-63 of each KV tile, 1: keys 64-127
+    // ============================================================ softmax (every other tile)
+    const int h = wg - 1;           // tiles j with j % 2 == h, in S buffer h
     const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const int grow = qt * kBlkQ + row;  // query index within the sequence
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t c0 = 64u * h;    // this half's S columns; its P8 takes the first 16
+    const uint32_t tS = tmem + lane_base + 128u * h;
+    const int rx = row & 7;
     bool ok = !dead;
     // this row's Q scale, and the K scales of the sequence; ksc32(j, c) is the scale of
     // keys 32c .. 32c + 31 of KV tile j (its 64-token block, or its own 32-token block)
-    const float sq = a.fine
+    const float sq = kFine
         ? a.q_scale[static_cast<int64_t>(hq) * seq.t_pad + off + qt * kBlkQ + row]
         : a.q_scale[static_cast<int64_t>(hq) * (seq.t_pad / kBlkQ) + off / kBlkQ + qt];
-    const int kblk = a.fine ? kBlkKFine : kBlkK;
+    constexpr int kblk = kFine ? kBlkKFine : kBlkK;
     const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kblk) + off / kblk;
-    auto ksc32 = [&](int j, int c) { return a.fine ? ksc[4 * j + c] : ksc[2 * j + (c >> 1)]; };
+    auto ksc32 = [&](int j, int c) { return kFine ? ksc[4 * j + c] : ksc[2 * j + (c >> 1)]; };
+    const double sq_sc = static_cast<double>(sq) * a.scale;  // q_scale sm_scale
 
-    // both S buffers start free
-    if (ok && lane == 0) { mbar_arrive(bar_sfree(0)); mbar_arrive(bar_sfree(1)); }
-
-    float m = -INFINITY, l = 0.0f;
-    for (int j = 0; j < nkv && ok; ++j) {
-      const int buf = j & 1;
-      const uint32_t tS = tmem + lane_base + 128u * buf;
-      // logit factors of this half's two 32-key chunks
-      const float cka = __fmul_rn(__fmul_rn(sq, ksc32(j, 2 * h)), a.scale_log2);
-      const float ckb = __fmul_rn(__fmul_rn(sq, ksc32(j, 2 * h + 1)), a.scale_log2);
+    float l = 0.0f;           // this warpgroup's partial sum, relative to mh
+    double mh = -INFINITY;    // the max of this warpgroup's last tile
+    for (int j = h; j < nkv && ok; j += 2) {
+      float sk[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) sk[c] = ksc32(j, c);
       const bool masked = (a.causal && j == qt) || (j + 1) * kKvTile > n;
-      const int kv0 = j * kKvTile + 64 * h;  // first key of this half
+      const int kv0 = j * kKvTile;  // first key of the tile
       auto dropped = [&](int key) { return key >= n || (a.causal && key > grow); };
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull(buf), (j >> 1) & 1, 0x301 + h));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull(h), (j >> 1) & 1, 0x301 + h));
       if (!ok) break;
       tc_fence_after();
 
-      // pass 1: the largest magic-offset score of this half (masked keys read as 0,
-      // below every valid value 12582912 + S)
-      uint32_t ra[32], rb[32];
-      tmem_ld32(tS + c0, ra);
-      tmem_ld32(tS + c0 + 32u, rb);
-      tmem_wait_ld_tied(ra, rb);
-      uint32_t keep_a = 0xFFFFFFFFu, keep_b = 0xFFFFFFFFu;
-      if (masked) {
-        keep_a = 0u;
-        keep_b = 0u;
+      uint32_t s[4][32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if (dropped(kv0 + i)) ra[i] = 0u; else keep_a |= 1u << i;
-          if (dropped(kv0 + 32 + i)) rb[i] = 0u; else keep_b |= 1u << i;
-        }
-      }
-      // this half's max logit (log2 units): each 32-key chunk's largest score times the
-      // chunk's factor (the same as the largest score of the half times its factor when
-      // both chunks share one K block: rounding is monotone)
-      const float hma = max32(ra, 0.0f), hmb = max32(rb, 0.0f);
-      const float hs = fmaxf(hma > 1.0e6f ? __fmul_rn(__fsub_rn(hma, kMagic), cka) : -INFINITY,
-                             hmb > 1.0e6f ? __fmul_rn(__fsub_rn(hmb, kMagic), ckb) : -INFINITY);
-      // exchange with the other softmax warp of this lane quarter
-      xchg[(buf * 2 + h) * 128 + row] = hs;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_xchg(buf, quarter));
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_xchg(buf, quarter), (j >> 1) & 1, 0x305 + h));
-      if (!ok) break;
-      const float mt = fmaxf(hs, xchg[(buf * 2 + (1 - h)) * 128 + row]);
-      const float m_new = fmaxf(m, mt);
-      const float alpha = ex2(m - m_new);
-      const float nbias = __fsub_rn(kLog2_448, m_new);
-      if (h == 0) alph[buf * 128 + row] = alpha;
-
-      // pass 2 on the same registers: p = 448 * 2^(u - m'), e4m3 P8 into this half's
-      // first 16 columns
-      f2 acc = make_float2(0.0f, 0.0f);
-      uint32_t w[8];
-      if (masked) p8_chunk<true>(ra, cka, nbias, acc, w, keep_a);
-      else p8_chunk<false>(ra, cka, nbias, acc, w, 0u);
-      tmem_st8(tS + c0, w);
-      if (masked) p8_chunk<true>(rb, ckb, nbias, acc, w, keep_b);
-      else p8_chunk<false>(rb, ckb, nbias, acc, w, 0u);
-      tmem_st8(tS + c0 + 8u, w);
-      l = l * alpha + (f2_lo(acc) + f2_hi(acc));
-      m = m_new;
-      tmem_wait_st();
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32u * c, s[c]);
+      tmem_wait_ld_tied(s[0]);
+      pin_regs(s[1]);
+      pin_regs(s[2]);
+      pin_regs(s[3]);
+      // S is in registers: the buffer may take S(j + 2)
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) { mbar_arrive(bar_pfull(buf)); mbar_arrive(bar_sfree(buf)); }
+      if (lane == 0) mbar_arrive(bar_sfree(h));
+
+      uint32_t keep[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
+      if (masked) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          keep[c] = 0u;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (dropped(kv0 + 32 * c + i)) s[c][i] = 0u; else keep[c] |= 1u << i;
+          }
+        }
+      }
+      // each chunk's largest score; the tile's max logit x = ((S q_scale) k_scale) sm_scale
+      // in fp64 (x is monotone in S within a chunk, so this is max_j x_j)
+      float hm[4];
+      double mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        hm[c] = max32(s[c]);
+        if (hm[c] > 1.0e6f) {
+          const double x = ((static_cast<double>(hm[c] - kMagic) * static_cast<double>(sq)) *
+                            static_cast<double>(sk[c])) * a.scale;
+          mt = fmax(mt, x);
+        }
+      }
+      // the running max after the previous tile comes from the other warpgroup
+      double m_prev = -INFINITY;
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_mready((j - 1) & 1), ((j - 1) >> 1) & 1, 0x303 + h));
+        if (!ok) break;
+        m_prev = mrun[((j - 1) & 1) * 128 + row];
+      }
+      const double m_new = fmax(m_prev, mt);
+      mrun[(j & 1) * 128 + row] = m_new;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_mready(j & 1));
+      // alpha = e^(m - m') for the correction warps (slot j % 4)
+      if (j >= kAlphaRing) {
+        const int jo = j - kAlphaRing;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_afree(jo % kAlphaRing), (jo / kAlphaRing) & 1, 0x305 + h));
+        if (!ok) break;
+      }
+      alph[(j % kAlphaRing) * 128 + row] = ex2(static_cast<float>((m_prev - m_new) * kLog2E64));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_afull(j % kAlphaRing));
+      // the P buffer of tile j was last read by PV(j - PB)
+      if (j >= PB) {
+        const int jo = j - PB;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_pfree(jo % PB), (jo / PB) & 1, 0x307 + h));
+        if (!ok) break;
+      }
+
+      // per chunk: c_c = q_scale k_scale_c sm_scale log2 e and
+      // nb_c = S_max_c c_c - m' log2 e + log2 ps, in fp64, each rounded once
+      const double ml = m_new * kLog2E64;
+      const uint32_t prow = sbase + L::kPOff + (j % PB) * L::kTileP + row * 128;
+      f2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const double cc = sq_sc * static_cast<double>(sk[c]) * kLog2E64;
+        const float ck = static_cast<float>(cc);
+        const float nb = hm[c] > 1.0e6f
+            ? static_cast<float>(static_cast<double>(hm[c] - kMagic) * cc - ml + kLog2Ps) : 0.0f;
+        ChunkExact ex{sq, sk[c], a.scale, m_new};
+        if (masked) p_chunk<PV, true, kExact>(s[c], hm[c], ck, nb, acc, keep[c], prow, rx, c, ex);
+        else p_chunk<PV, false, kExact>(s[c], hm[c], ck, nb, acc, 0u, prow, rx, c, ex);
+      }
+      l = l * ex2(static_cast<float>((mh - m_new) * kLog2E64)) + (acc.x + acc.y);
+      mh = m_new;
+      fence_proxy_async_smem();  // P stores -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_pfull(j % PB));
     }
-    // hand the row's partial sum (and, from the first half, its max) to the epilogue
+    // hand the row's partial sum, and the max it is relative to, to the epilogue
     lfin[h * 128 + row] = l;
-    if (h == 0) lfin[256 + row] = m;
+    mfin[h * 128 + row] = mh;
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_epi);
   } else {
@@ -542,18 +692,16 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const uint32_t tO = tmem + lane_base + kColO;
     bool ok = !dead;
 
-    // both S buffers start free
-    if (ok && lane == 0) { mbar_arrive(bar_sfree(0)); mbar_arrive(bar_sfree(1)); }
-
     for (int j = 0; j < nkv && ok; ++j) {
-      const int buf = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait<true>(bar_pfull(buf), (j >> 1) & 1, 0x401)) &&
-           __all_sync(0xffffffffu, mbar_wait<true>(bar_pvfull, j & 1, 0x402));
+      const int sa = j % kAlphaRing;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_afull(sa), (j / kAlphaRing) & 1, 0x401)) &&
+           __all_sync(0xffffffffu, mbar_wait(bar_pvfull, j & 1, 0x402));
       if (!ok) break;
       tc_fence_after();
-      // PV(j) has read P8(j): buffer j % 2 may take S(j + 2)
-      if (lane == 0) mbar_arrive(bar_sfree(buf));
-      const f2 al = make_float2(alph[buf * 128 + row], alph[buf * 128 + row]);
+      const float al = alph[sa * 128 + row];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_afree(sa));
+      const f2 AL = make_float2(al, al);
       // O = alpha * O + PV_blk, 32 columns at a time (the first tile just copies PV_blk)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -561,32 +709,41 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         tmem_ld32(tPV + 32u * c, rp);
         if (j > 0) {
           tmem_ld32(tO + 32u * c, ro);
-          tmem_wait_ld_tied(rp, ro);
+          tmem_wait_ld_tied(rp);
+          pin_regs(ro);
+        } else {
+          tmem_wait_ld_tied(rp);
+        }
+        if (c == D / 32 - 1) {  // the whole PV block has been read: PV(j + 1) may run
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_pvfree);
+        }
+        if (j > 0) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const f2 o = f2_fma(pair_of(ro, i), al, pair_of(rp, i));
+            const f2 o = f2_fma(pair_of(ro, i), AL, pair_of(rp, i));
             ro[2 * i] = __float_as_uint(o.x);
             ro[2 * i + 1] = __float_as_uint(o.y);
           }
           tmem_st32(tO + 32u * c, ro);
         } else {
-          tmem_wait_ld_tied(rp);
           tmem_st32(tO + 32u * c, rp);
         }
       }
-      // PV_blk has been read and O written back: the next PV may overwrite PV_blk
       tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_pvfree);
     }
 
     // ---------------------------------------------------------------- epilogue
-    ok = ok && __all_sync(0xffffffffu, mbar_wait(bar_epi, 0, 0x403));
+    ok = ok && __all_sync(0xffffffffu, mbar_wait<true>(bar_epi, 0, 0x403));
     if (ok) {
       tc_fence_after();
-      const float l = lfin[row] + lfin[128 + row];
-      const float m = lfin[256 + row];
+      // the two warpgroups' sums are relative to the max of their own last tile;
+      // the overall max is that of the last tile
+      const double m0 = mfin[row], m1 = mfin[128 + row];
+      const double m = fmax(m0, m1);
+      const float l = lfin[row] * ex2(static_cast<float>((m0 - m) * kLog2E64)) +
+                      lfin[128 + row] * ex2(static_cast<float>((m1 - m) * kLog2E64));
       const float inv_l = 1.0f / l;
       const float* vs = a.v_scale + (static_cast<int64_t>(b) * a.hkv + hk) * D;
       const int64_t orow =
@@ -599,7 +756,10 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         if (grow < n) {
           float v[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ro[i]) * vs[32 * c + i] * inv_l;
+          for (int i = 0; i < 32; ++i) {
+            const float sv = PV == kPvE4m3 ? vs[32 * c + i] : 1.0f;
+            v[i] = __uint_as_float(ro[i]) * sv * inv_l;
+          }
           if (a.out_dtype == 2) {
             float* dst = reinterpret_cast<float*>(a.out) + orow + 32 * c;
 #pragma unroll
@@ -628,7 +788,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       }
       if (a.lse != nullptr && grow < n)
         a.lse[static_cast<int64_t>(hq) * seq.t_pad + off + grow] =
-            m * 0.6931471805599453f + (logf(l) - kLn448);
+            static_cast<float>(m) + (logf(l) - kLnPs);
     }
   }
 

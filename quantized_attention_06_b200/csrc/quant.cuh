@@ -15,6 +15,8 @@
 //   v_finalize per (sequence, kv head): vmax, v_scale = vmax / 448
 //   quant_qk   Q blocks of 128 tokens and smoothed K blocks of 64 tokens -> int8 + scale
 //   quant_v    V -> e4m3 with per-channel scale, written token-contiguous (transposed)
+//   transpose_v16  V kept in its 16-bit input type, written token-contiguous (the
+//              16-bit PV option), and fill_ones for its unit V scales
 #pragma once
 
 #include "sage_device.cuh"
@@ -374,6 +376,69 @@ quant_v_kernel(const __grid_constant__ Seq seq, const __grid_constant__ VQuantAr
     const uint4 w = *reinterpret_cast<const uint4*>(tile + ch * kPad + ((j ^ (ch & 7)) << 4));
     *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(ch) * seq.t_pad + j * 16) = w;
   }
+}
+
+// ------------------------------------------------------------------------- V 16-bit
+// The 16-bit PV option keeps V at its input values: the same token-contiguous
+// [Hkv][D][T_pad] layout as the e4m3 codes, two bytes per entry.  One CTA: one
+// 128-token block of one KV head; thread (cg, tg) holds channels 8cg .. 8cg+7 of
+// tokens TPT*tg .. TPT*tg+TPT-1 and writes each channel's TPT values as one word into
+// a [D][128] tile whose 16-byte chunks are XOR-swizzled by channel; the rows then
+// leave as 16-byte stores.
+template <typename T, int D, class Seq>
+__global__ void __launch_bounds__(kQuantThreads)
+transpose_v16_kernel(const __grid_constant__ Seq seq, const __grid_constant__ VQuantArgs a) {
+  constexpr int CG = D / 8;
+  constexpr int TG = kQuantThreads / CG;
+  constexpr int TPT = kPad / TG;  // 8 (d = 128) or 4 (d = 64)
+  static_assert(TPT == 4 || TPT == 8, "tile shape");
+  __shared__ __align__(16) uint8_t tile[D * kPad * 2];  // D rows of 256 bytes
+  const int pb = blockIdx.x, h = blockIdx.y;
+  const SeqPos sp = locate(seq, pb * kPad, a.sb, a.st);
+  const int t0 = pb * kPad - sp.off;
+  const int cg = threadIdx.x % CG, tg = threadIdx.x / CG;
+  const T* src = reinterpret_cast<const T*>(a.v) + sp.base + h * a.sh + cg * 8;
+  uint32_t raw[TPT][4];  // token u: channels 8cg .. 8cg+7 as 8 x 16 bits
+#pragma unroll
+  for (int u = 0; u < TPT; ++u) {
+    const int t = t0 + TPT * tg + u;
+    const uint4 x = (t < sp.n) ? ld_stream16(src + static_cast<int64_t>(t) * a.st) : make_uint4(0, 0, 0, 0);
+    raw[u][0] = x.x; raw[u][1] = x.y; raw[u][2] = x.z; raw[u][3] = x.w;
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int c = (k + cg) & 7;  // rotated by cg: fewer threads of a warp on one bank
+    const int ch = cg * 8 + c;
+    const int tok = TPT * tg;
+    uint32_t w[TPT / 2];
+#pragma unroll
+    for (int u = 0; u < TPT; u += 2) {
+      uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {  // no dynamically indexed register array
+        if (cc == c) {
+          lo = (raw[u][cc >> 1] >> (16 * (cc & 1))) & 0xFFFFu;
+          hi = (raw[u + 1][cc >> 1] >> (16 * (cc & 1))) & 0xFFFFu;
+        }
+      }
+      w[u / 2] = lo | (hi << 16);
+    }
+    const int off = ch * (kPad * 2) + ((((tok >> 3) ^ ch) & 15) << 4) + (tok & 7) * 2;
+    if constexpr (TPT == 8) *reinterpret_cast<uint4*>(tile + off) = make_uint4(w[0], w[1], w[2], w[3]);
+    else *reinterpret_cast<uint2*>(tile + off) = make_uint2(w[0], w[1]);
+  }
+  __syncthreads();
+  uint8_t* dst = reinterpret_cast<uint8_t*>(a.v8) + (static_cast<int64_t>(h) * D * seq.t_pad + pb * kPad) * 2;
+  for (int i = threadIdx.x; i < D * 16; i += kQuantThreads) {
+    const int ch = i >> 4, j = i & 15;
+    const uint4 w = *reinterpret_cast<const uint4*>(tile + ch * (kPad * 2) + (((j ^ ch) & 15) << 4));
+    *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(ch) * seq.t_pad * 2 + j * 16) = w;
+  }
+}
+
+__global__ void fill_ones_kernel(float* __restrict__ x, int64_t n) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) x[i] = 1.0f;
 }
 
 }  // namespace sage

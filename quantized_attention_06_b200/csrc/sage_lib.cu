@@ -7,6 +7,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <type_traits>
 
@@ -14,6 +15,7 @@
 #include "attn_fwd.cuh"
 #include "debug_qk.cuh"
 #include "quant.cuh"
+#include "quant_fused.cuh"
 #include "sage_device.cuh"
 #include "seq_table.cuh"
 
@@ -42,6 +44,7 @@ sage_status_t plan(const sage_problem_t* p, Layout& L, SeqVarlen* storage) {
   if (p->dtype != SAGE_FP16 && p->dtype != SAGE_BF16) return SAGE_ERR_UNSUPPORTED;
   if (p->granularity != SAGE_GRAN_BLOCK && p->granularity != SAGE_GRAN_THREAD)
     return SAGE_ERR_INVALID_ARGUMENT;
+  if (p->pv != SAGE_PV_FP8 && p->pv != SAGE_PV_FP16) return SAGE_ERR_INVALID_ARGUMENT;
   L.nseq = p->batch;
   if (p->cu_seqlens_host == nullptr) {
     if (p->seqlen < 1) return SAGE_ERR_INVALID_ARGUMENT;
@@ -97,13 +100,20 @@ bool strides_ok(const sage_problem_t* p, const int64_t s[3], int elem_bytes) {
   return true;
 }
 
-sage_status_t device_ok() {
+// The current device must be an sm_100 part, and `stream` must belong to it: the
+// kernels run on the current device, so a stream of another device would make them
+// dereference that device's pointers.
+sage_status_t device_ok(sage_stream_t stream) {
   int dev = 0, major = 0, minor = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
     return SAGE_ERR_CUDA;
-  return (major == 10 && minor == 0) ? SAGE_OK : SAGE_ERR_UNSUPPORTED;
+  if (major != 10 || minor != 0) return SAGE_ERR_UNSUPPORTED;
+  int sdev = -1;
+  if (cudaStreamGetDevice(reinterpret_cast<cudaStream_t>(stream), &sdev) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  return sdev == dev ? SAGE_OK : SAGE_ERR_INVALID_ARGUMENT;
 }
 
 sage_status_t launched() {
@@ -172,6 +182,14 @@ sage_status_t launch_quant_v(const Seq& seq, const sage_problem_t* p, int64_t t_
                              const int64_t* vs, uint8_t* v8, float* v_scale, void* ws,
                              cudaStream_t st) {
   const int nblk = static_cast<int>(t_pad / kPad);
+  if (p->pv == SAGE_PV_FP16) {  // V keeps its 16-bit values, transposed; unit scales
+    VQuantArgs a{};
+    a.v = v; a.sb = vs[0]; a.sh = vs[1]; a.st = vs[2]; a.v8 = v8; a.hkv = p->heads_kv;
+    transpose_v16_kernel<T, D, Seq><<<dim3(nblk, p->heads_kv), kQuantThreads, 0, st>>>(seq, a);
+    const int64_t ns = static_cast<int64_t>(p->batch) * p->heads_kv * D;
+    fill_ones_kernel<<<static_cast<unsigned>((ns + 255) / 256), 256, 0, st>>>(v_scale, ns);
+    return launched();
+  }
   float* partial = reinterpret_cast<float*>(ws);
   float* vmax = partial + static_cast<size_t>(p->heads_kv) * nblk * D;
   v_colmax_kernel<T, D, Seq><<<dim3(nblk, p->heads_kv), kQuantThreads, 0, st>>>(
@@ -184,21 +202,104 @@ sage_status_t launch_quant_v(const Seq& seq, const sage_problem_t* p, int64_t t_
   return launched();
 }
 
-template <int D, class Seq>
+template <int D, class Seq, bool kFine, int PV>
 sage_status_t launch_attn(const Seq& seq, int64_t ncta, const CUtensorMap& mq, const CUtensorMap& mk,
                           const CUtensorMap& mv, const AttnArgs& a, cudaStream_t st) {
-  auto kern = sage_attn_fwd_kernel<D, Seq>;
+  auto kern = sage_attn_fwd_kernel<D, Seq, kFine, PV>;
   // the warpgroups trade registers with setmaxnreg; the split only adds up if the
   // kernel was compiled to exactly the launch allocation it assumes
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SAGE_ERR_CUDA;
   if (fa.numRegs != kAttnLaunchRegs || fa.maxThreadsPerBlock < kAttnThreads) return SAGE_ERR_UNSUPPORTED;
-  const size_t smem = std::max(static_cast<size_t>(AttnSmem<D>::kAlloc), kMinAttnSmem);
+  const size_t smem = std::max(static_cast<size_t>(AttnCfg<D, PV>::kAlloc), kMinAttnSmem);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return SAGE_ERR_CUDA;
   kern<<<static_cast<unsigned>(ncta), kAttnThreads, smem, st>>>(mq, mk, mv, seq, a);
   return launched();
+}
+
+// Template dispatch of the attention kernel: head dim, granularity, PV format.
+template <class Seq>
+sage_status_t dispatch_attn(const Seq& seq, int64_t ncta, int d, bool fine, int pv,
+                            const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const AttnArgs& a, cudaStream_t st) {
+#define SAGE_ATTN(DD, FF, PP) \
+  if (d == DD && fine == FF && pv == PP) return launch_attn<DD, Seq, FF, PP>(seq, ncta, mq, mk, mv, a, st)
+  SAGE_ATTN(128, false, kPvE4m3); SAGE_ATTN(128, true, kPvE4m3);
+  SAGE_ATTN(64, false, kPvE4m3);  SAGE_ATTN(64, true, kPvE4m3);
+  SAGE_ATTN(128, false, kPvF16);  SAGE_ATTN(128, true, kPvF16);
+  SAGE_ATTN(64, false, kPvF16);   SAGE_ATTN(64, true, kPvF16);
+  SAGE_ATTN(128, false, kPvBf16); SAGE_ATTN(128, true, kPvBf16);
+  SAGE_ATTN(64, false, kPvBf16);  SAGE_ATTN(64, true, kPvBf16);
+#undef SAGE_ATTN
+  return SAGE_ERR_UNSUPPORTED;
+}
+
+// 4-D 16-bit tensor map over an input (d, tokens, heads, batch): the three outer
+// dimensions in ascending stride order, boxes of 64 channels x 128 tokens (128-byte
+// swizzle).  Reports where the token, head and batch dimensions landed.
+bool make_input_map(CUtensorMap* m, const void* base, const sage_problem_t* p, int heads,
+                    const int64_t s[3], int64_t ntok, int* dim_tok, int* dim_head, int* dim_batch) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const bool dense = p->cu_seqlens_host == nullptr;
+  struct Dim { uint64_t size, stride; int kind; } dm[3];
+  dm[0] = {static_cast<uint64_t>(ntok), static_cast<uint64_t>(s[2]) * 2, 0};
+  dm[1] = {static_cast<uint64_t>(heads), static_cast<uint64_t>(s[1]) * 2, 1};
+  if (dense) {
+    dm[2] = {static_cast<uint64_t>(p->batch), static_cast<uint64_t>(s[0]) * 2, 2};
+  } else {  // packed sequences: a unit batch dimension beyond the whole tensor
+    const uint64_t ext = std::max(dm[0].size * dm[0].stride, dm[1].size * dm[1].stride);
+    dm[2] = {1, round_up(ext, 16), 2};
+  }
+  std::sort(dm, dm + 3, [](const Dim& x, const Dim& y) { return x.stride < y.stride; });
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(p->head_dim), dm[0].size, dm[1].size, dm[2].size};
+  cuuint64_t strides[3] = {dm[0].stride, dm[1].stride, dm[2].stride};
+  cuuint32_t box[4] = {64, 1, 1, 1}, estr[4] = {1, 1, 1, 1};
+  for (int i = 0; i < 3; ++i) {
+    if (dm[i].kind == 0) { *dim_tok = i + 1; box[i + 1] = kPad; }
+    if (dm[i].kind == 1) *dim_head = i + 1;
+    if (dm[i].kind == 2) *dim_batch = i + 1;
+  }
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int D, class Seq>
+sage_status_t launch_quant_fused(const Seq& seq, const CUtensorMap& mq, const CUtensorMap& mk,
+                                 const CUtensorMap& mv, const FusedQuantArgs& a, cudaStream_t st) {
+  auto kern = quant_fused_kernel<T, D, Seq>;
+  const int smem = FusedCfg<D>::kAlloc;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  int dev = 0, nsm = 0, coop = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFusedThreads, smem) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  if (!coop || per_sm < 1) return SAGE_ERR_UNSUPPORTED;
+  void* args[] = {const_cast<CUtensorMap*>(&mq), const_cast<CUtensorMap*>(&mk),
+                  const_cast<CUtensorMap*>(&mv), const_cast<Seq*>(&seq),
+                  const_cast<FusedQuantArgs*>(&a)};
+  if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kern), dim3(nsm), dim3(kFusedThreads), args,
+                                  smem, st) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  return launched();
+}
+
+// Template dispatch: head dim, granularity, PV format (the sequence table type is the caller's).
+template <class Seq>
+sage_status_t dispatch_quant_fused(const Seq& seq, const sage_problem_t* p, const CUtensorMap& mq,
+                                   const CUtensorMap& mk, const CUtensorMap& mv,
+                                   const FusedQuantArgs& a, cudaStream_t st) {
+  if (p->dtype == SAGE_FP16)
+    return p->head_dim == 128 ? launch_quant_fused<__half, 128>(seq, mq, mk, mv, a, st)
+                              : launch_quant_fused<__half, 64>(seq, mq, mk, mv, a, st);
+  return p->head_dim == 128 ? launch_quant_fused<__nv_bfloat16, 128>(seq, mq, mk, mv, a, st)
+                            : launch_quant_fused<__nv_bfloat16, 64>(seq, mq, mk, mv, a, st);
 }
 
 }  // namespace
@@ -231,11 +332,17 @@ sage_status_t sage_buffer_sizes(const sage_problem_t* p, sage_sizes_t* sz) {
   sz->k8 = static_cast<size_t>(p->heads_kv) * tp * d;
   sz->k_scale = static_cast<size_t>(p->heads_kv) * (tp / (fine ? kBlkKFine : kBlkK)) * sizeof(float);
   sz->k_mean = static_cast<size_t>(p->batch) * p->heads_kv * d * sizeof(float);
-  sz->v8 = static_cast<size_t>(p->heads_kv) * d * tp;
+  const bool pv16 = p->pv == SAGE_PV_FP16;
+  sz->v8 = static_cast<size_t>(p->heads_kv) * d * tp * (pv16 ? 2 : 1);
   sz->v_scale = sz->k_mean;
   sz->workspace_qk = static_cast<size_t>(p->heads_kv) * (tp / kPad) * d * sizeof(double);
-  sz->workspace_v = static_cast<size_t>(p->heads_kv) * (tp / kPad) * d * sizeof(float) +
-                    static_cast<size_t>(p->batch) * p->heads_kv * d * sizeof(float);
+  sz->workspace_v = pv16 ? 0
+                         : static_cast<size_t>(p->heads_kv) * (tp / kPad) * d * sizeof(float) +
+                               static_cast<size_t>(p->batch) * p->heads_kv * d * sizeof(float);
+  // fused: fp64 K partial sums, fp32 V partial maxima, fp32 vmax (offsets 256-aligned)
+  sz->workspace_qkv = round_up(sz->workspace_qk, 256) +
+                      round_up(static_cast<size_t>(p->heads_kv) * (tp / kPad) * d * sizeof(float), 256) +
+                      static_cast<size_t>(p->batch) * p->heads_kv * d * sizeof(float);
   return SAGE_OK;
 }
 
@@ -255,7 +362,7 @@ sage_status_t sage_quant_qk(const sage_problem_t* p, const void* q, const int64_
     return SAGE_ERR_INVALID_ARGUMENT;
   if (!strides_ok(p, q_strides, 2) || !strides_ok(p, k_strides, 2)) return SAGE_ERR_INVALID_ARGUMENT;
   if (workspace_bytes < sz.workspace_qk) return SAGE_ERR_INVALID_ARGUMENT;
-  if ((st = device_ok()) != SAGE_OK) return st;
+  if ((st = device_ok(stream)) != SAGE_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 #define SAGE_QK(T, D)                                                                           \
   return L.varlen ? launch_quant_qk<T, D>(*L.var, p, L.t_pad, q, q_strides, k, k_strides, q8,    \
@@ -279,11 +386,11 @@ sage_status_t sage_quant_v(const sage_problem_t* p, const void* v, const int64_t
   if (st != SAGE_OK) return st;
   sage_sizes_t sz;
   sage_buffer_sizes(p, &sz);
-  if (!v || !v8 || !v_scale || !workspace) return SAGE_ERR_INVALID_ARGUMENT;
+  if (!v || !v8 || !v_scale || (!workspace && sz.workspace_v > 0)) return SAGE_ERR_INVALID_ARGUMENT;
   if (!aligned16(v) || !aligned16(v8) || !aligned16(workspace)) return SAGE_ERR_INVALID_ARGUMENT;
   if (!strides_ok(p, v_strides, 2)) return SAGE_ERR_INVALID_ARGUMENT;
   if (workspace_bytes < sz.workspace_v) return SAGE_ERR_INVALID_ARGUMENT;
-  if ((st = device_ok()) != SAGE_OK) return st;
+  if ((st = device_ok(stream)) != SAGE_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 #define SAGE_V(T, D)                                                                             \
   return L.varlen ? launch_quant_v<T, D>(*L.var, p, L.t_pad, v, v_strides, v8, v_scale, workspace, s) \
@@ -294,6 +401,59 @@ sage_status_t sage_quant_v(const sage_problem_t* p, const void* v, const int64_t
     if (p->head_dim == 128) { SAGE_V(__nv_bfloat16, 128); } else { SAGE_V(__nv_bfloat16, 64); }
   }
 #undef SAGE_V
+}
+
+sage_status_t sage_quant_qkv(const sage_problem_t* p, const void* q, const int64_t q_strides[3],
+                             const void* k, const int64_t k_strides[3], const void* v,
+                             const int64_t v_strides[3], int8_t* q8, float* q_scale, int8_t* k8,
+                             float* k_scale, float* k_mean, void* v8, float* v_scale,
+                             void* workspace, size_t workspace_bytes, sage_stream_t stream) {
+  static thread_local SeqVarlen var;
+  Layout L;
+  sage_status_t st = plan(p, L, &var);
+  if (st != SAGE_OK) return st;
+  sage_sizes_t sz;
+  sage_buffer_sizes(p, &sz);
+  if (!q || !k || !v || !q8 || !q_scale || !k8 || !k_scale || !k_mean || !v8 || !v_scale || !workspace)
+    return SAGE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q8) || !aligned16(k8) ||
+      !aligned16(v8) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return SAGE_ERR_INVALID_ARGUMENT;
+  if (!strides_ok(p, q_strides, 2) || !strides_ok(p, k_strides, 2) || !strides_ok(p, v_strides, 2))
+    return SAGE_ERR_INVALID_ARGUMENT;
+  const bool dense = p->cu_seqlens_host == nullptr;
+  for (const int64_t* s3 : {q_strides, k_strides, v_strides})
+    for (int i = dense ? 0 : 1; i < 3; ++i)
+      if (s3[i] < p->head_dim) return SAGE_ERR_INVALID_ARGUMENT;
+  if (workspace_bytes < sz.workspace_qkv) return SAGE_ERR_INVALID_ARGUMENT;
+  if ((st = device_ok(stream)) != SAGE_OK) return st;
+  const int64_t ntok = dense ? p->seqlen : p->cu_seqlens_host[p->batch];
+  FusedQuantArgs a{};
+  CUtensorMap mq, mk, mv;
+  int dt = 0, dh = 0, db = 0, dt2 = 0, dh2 = 0, db2 = 0, dt3 = 0, dh3 = 0, db3 = 0;
+  if (!make_input_map(&mq, q, p, p->heads_q, q_strides, ntok, &dt, &dh, &db) ||
+      !make_input_map(&mk, k, p, p->heads_kv, k_strides, ntok, &dt2, &dh2, &db2) ||
+      !make_input_map(&mv, v, p, p->heads_kv, v_strides, ntok, &dt3, &dh3, &db3))
+    return SAGE_ERR_CUDA;
+  // the kernel addresses all three maps with one coordinate order
+  if (dt != dt2 || dt != dt3 || dh != dh2 || dh != dh3 || db != db2 || db != db3)
+    return SAGE_ERR_INVALID_ARGUMENT;
+  a.dim_tok = dt; a.dim_head = dh; a.dim_batch = db;
+  a.q8 = q8; a.q_scale = q_scale; a.k8 = k8; a.k_scale = k_scale; a.k_mean = k_mean;
+  a.v8 = v8; a.v_scale = v_scale;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.ksum = reinterpret_cast<double*>(ws);
+  ws += round_up(sz.workspace_qk, 256);
+  a.vpart = reinterpret_cast<float*>(ws);
+  ws += round_up(static_cast<size_t>(p->heads_kv) * (L.t_pad / kPad) * p->head_dim * sizeof(float), 256);
+  a.vmax = reinterpret_cast<float*>(ws);
+  a.hq = p->heads_q; a.hkv = p->heads_kv; a.nblk = static_cast<int>(L.t_pad / kPad);
+  a.batch = p->batch;
+  a.fine = p->granularity == SAGE_GRAN_THREAD ? 1 : 0;
+  a.pv16 = p->pv == SAGE_PV_FP16 ? 1 : 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return L.varlen ? dispatch_quant_fused(*L.var, p, mq, mk, mv, a, s)
+                  : dispatch_quant_fused(L.dense, p, mq, mk, mv, a, s);
 }
 
 sage_status_t sage_attn_fwd(const sage_problem_t* p, const int8_t* q8, const float* q_scale,
@@ -312,13 +472,15 @@ sage_status_t sage_attn_fwd(const sage_problem_t* p, const int8_t* q8, const flo
     return SAGE_ERR_UNSUPPORTED;
   if (!strides_ok(p, out_strides, out_dtype == SAGE_FP32 ? 4 : 2)) return SAGE_ERR_INVALID_ARGUMENT;
   if (!(sm_scale == sm_scale) || std::isinf(sm_scale)) return SAGE_ERR_INVALID_ARGUMENT;
-  if ((st = device_ok()) != SAGE_OK) return st;
+  if ((st = device_ok(stream)) != SAGE_OK) return st;
   const int d = p->head_dim;
   const uint64_t tp = static_cast<uint64_t>(L.t_pad);
+  const bool pv16 = p->pv == SAGE_PV_FP16;
+  const uint64_t vrow = tp * (pv16 ? 2 : 1);  // bytes per V^T row
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q8, d, tp * p->heads_q, d, d, kBlkQ, qk_swizzle(d)) ||
       !make_map(&mk, k8, d, tp * p->heads_kv, d, d, kKvTile, qk_swizzle(d)) ||
-      !make_map(&mv, v8, tp, static_cast<uint64_t>(p->heads_kv) * d, tp, kKvTile, d,
+      !make_map(&mv, v8, vrow, static_cast<uint64_t>(p->heads_kv) * d, vrow, 128, d,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return SAGE_ERR_CUDA;
   AttnArgs a{};
@@ -327,21 +489,20 @@ sage_status_t sage_attn_fwd(const sage_problem_t* p, const int8_t* q8, const flo
   a.osb = out_strides[0]; a.osh = out_strides[1]; a.ost = out_strides[2];
   a.lse = lse;
   a.hq = p->heads_q; a.hkv = p->heads_kv; a.group = p->heads_q / p->heads_kv;
-  const float scale = sm_scale > 0.0f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(d));
-  a.scale_log2 = scale * kLog2E;
+  // fp64, as the definition forms the logits: 1/sqrt(d) unless the caller gives one
+  a.scale = sm_scale > 0.0f ? static_cast<double>(sm_scale) : 1.0 / std::sqrt(static_cast<double>(d));
   a.causal = is_causal ? 1 : 0;
-  a.fine = p->granularity == SAGE_GRAN_THREAD ? 1 : 0;
+  const bool fine = p->granularity == SAGE_GRAN_THREAD;
+  const int pv = !pv16 ? kPvE4m3 : (p->dtype == SAGE_BF16 ? kPvBf16 : kPvF16);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (L.varlen) {
     const int64_t ncta = L.var->cta[p->batch];
     if (ncta == 0) return SAGE_OK;
-    return d == 128 ? launch_attn<128>(*L.var, ncta, mq, mk, mv, a, s)
-                    : launch_attn<64>(*L.var, ncta, mq, mk, mv, a, s);
+    return dispatch_attn(*L.var, ncta, d, fine, pv, mq, mk, mv, a, s);
   }
   const int64_t tiles = (L.dense.len + kBlkQ - 1) / kBlkQ;
   const int64_t ncta = static_cast<int64_t>(p->batch) * p->heads_q * tiles;
-  return d == 128 ? launch_attn<128>(L.dense, ncta, mq, mk, mv, a, s)
-                  : launch_attn<64>(L.dense, ncta, mq, mk, mv, a, s);
+  return dispatch_attn(L.dense, ncta, d, fine, pv, mq, mk, mv, a, s);
 }
 
 sage_status_t sage_debug_qk_int32(const sage_problem_t* p, const int8_t* q8, const int8_t* k8,
@@ -354,7 +515,7 @@ sage_status_t sage_debug_qk_int32(const sage_problem_t* p, const int8_t* q8, con
     return SAGE_ERR_INVALID_ARGUMENT;
   if (seq < 0 || seq >= p->batch || head_q < 0 || head_q >= p->heads_q)
     return SAGE_ERR_INVALID_ARGUMENT;
-  if ((st = device_ok()) != SAGE_OK) return st;
+  if ((st = device_ok(stream)) != SAGE_OK) return st;
   const int d = p->head_dim;
   const int n = L.varlen ? L.var->cu[seq + 1] - L.var->cu[seq] : L.dense.len;
   const int off = L.varlen ? L.var->poff[seq] : seq * L.dense.pad_len;
@@ -382,7 +543,7 @@ sage_status_t sage_debug_qk_int32(const sage_problem_t* p, const int8_t* q8, con
 
 sage_status_t sage_debug_watchdog_selftest(unsigned int limit_us, sage_stream_t stream) {
   if (limit_us == 0 || limit_us > 1000000u) return SAGE_ERR_INVALID_ARGUMENT;
-  sage_status_t st = device_ok();
+  sage_status_t st = device_ok(stream);
   if (st != SAGE_OK) return st;
   watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<uint64_t>(limit_us) * 1000ull);
@@ -459,7 +620,7 @@ extern "C" sage_status_t sage_quant_qk_noalloc(const sage_problem_t* p, const vo
     return SAGE_ERR_INVALID_ARGUMENT;
   if (!strides_ok(p, q_strides, 2) || !strides_ok(p, k_strides, 2)) return SAGE_ERR_INVALID_ARGUMENT;
   if (sz.workspace_qk > SAGE_NOALLOC_SCRATCH_BYTES) return SAGE_ERR_TOO_LARGE;
-  if ((st = device_ok()) != SAGE_OK) return st;
+  if ((st = device_ok(stream)) != SAGE_OK) return st;
   void* ws = nullptr;
   if ((st = static_scratch(&ws)) != SAGE_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -606,8 +767,11 @@ extern "C" sage_status_t sage_attn_host(const sage_problem_t* p, int tensor_layo
   const sage_problem_t cfull = chunk_problem(p, hc);
   Slot slot[2];
   if (!carve_slot(cfull, out_dtype, nullptr, &slot[0])) return SAGE_ERR_INVALID_ARGUMENT;
-  if (workspace_bytes < 2 * slot[0].bytes) return SAGE_ERR_INVALID_ARGUMENT;
-  if ((st = device_ok()) != SAGE_OK) return st;
+  // every slot is as large as a full chunk needs; a short last chunk must not move
+  // the base of the next slot
+  const size_t slot_bytes = slot[0].bytes;
+  if (workspace_bytes < 2 * slot_bytes) return SAGE_ERR_INVALID_ARGUMENT;
+  if ((st = device_ok(stream)) != SAGE_OK) return st;
 
   std::lock_guard<std::mutex> lock(g_pipe_mu);
   HostPipe* P = nullptr;
@@ -652,7 +816,7 @@ extern "C" sage_status_t sage_attn_host(const sage_problem_t* p, int tensor_layo
       const int heads = (p->heads_kv - h0 < hc) ? p->heads_kv - h0 : hc;
       const sage_problem_t cp = chunk_problem(p, heads);
       const int i = c & 1;
-      carve_slot(cp, out_dtype, static_cast<uint8_t*>(workspace) + i * slot[0].bytes, &slot[i]);
+      carve_slot(cp, out_dtype, static_cast<uint8_t*>(workspace) + i * slot_bytes, &slot[i]);
       Slot& S = slot[i];
       // copy-in: the slot's inputs are free once chunk c-2's kernels are done
       if (c >= 2 && cudaStreamWaitEvent(P->h2d, P->k_done[i], 0) != cudaSuccess) return SAGE_ERR_CUDA;

@@ -55,18 +55,33 @@ def padded_offsets(lens):
     return offs, o
 
 
+def oracle_pv(pv: str, dtype: str) -> str:
+    """The oracle's PV format for the library's: e4m3, or the input's 16-bit type."""
+    return "e4m3" if pv == "fp8" else dtype
+
+
 def run_gpu(x: dict, dtype: str, layout: str, varlen: bool, causal: bool, out_dtype=torch.float32,
-            return_lse=True):
+            return_lse=True, pv="fp8", granularity="block"):
     q = to_device(x["q"], dtype, layout, varlen)
     k = to_device(x["k"], dtype, layout, varlen)
     v = to_device(x["v"], dtype, layout, varlen)
     cu = x["cu_seqlens"] if varlen else None
-    z = api.quant_qk(q, k, layout, cu)
+    z = api.quant_qk(q, k, layout, cu, granularity=granularity, pv=pv)
     api.quant_v(v, z)
     out, lse = api.attn_fwd(z, is_causal=causal, out_dtype=out_dtype, return_lse=True)
     torch.cuda.synchronize()
     assert api.poll_device_status() == 0
     return z, out, lse
+
+
+def reference_rows(q, k, v, rows, causal):
+    """Full-precision softmax attention (fp64, no quantization) for the given query rows."""
+    x = (q[rows].astype(np.float64) @ k.astype(np.float64).T) / np.sqrt(q.shape[1])
+    if causal:
+        x = np.where(np.arange(k.shape[0])[None, :] > np.asarray(rows)[:, None], -np.inf, x)
+    x = x - x.max(axis=1, keepdims=True)
+    p = np.exp(x)
+    return (p @ v.astype(np.float64)) / p.sum(axis=1, keepdims=True)
 
 
 def metrics(a: np.ndarray, b: np.ndarray):

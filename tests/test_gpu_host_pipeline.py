@@ -50,3 +50,15 @@ def test_host_path_back_to_back_and_stream_order():
     torch.cuda.current_stream().synchronize()
     assert torch.equal(o1, r1) and torch.equal(o2, r2)
     assert api.poll_device_status() == 0
+
+
+@pytest.mark.parametrize("chunk", [3, 0])
+def test_host_path_short_chunk_in_slot_zero(chunk):
+    # Hkv = 8 in chunks of 3 gives chunks of 3, 3, 2 per batch entry; with B = 3 the
+    # short chunk lands in slot 0 as well as slot 1.  Every slot must keep the full
+    # chunk's size as its stride, or a later chunk's buffers overlap one still in flight.
+    q, k, v = _inputs(3, 16, 8, 257, 128, torch.bfloat16, "NHD", 31)
+    ref = api.sageattn(q.cuda(), k.cuda(), v.cuda(), tensor_layout="NHD").cpu()
+    out = api.sageattn_host(q, k, v, tensor_layout="NHD", kv_heads_per_chunk=chunk)
+    assert torch.equal(out, ref)
+    assert api.poll_device_status() == 0
