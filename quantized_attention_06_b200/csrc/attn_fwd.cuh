@@ -8,23 +8,23 @@
 // compatible online softmax).
 //
 // CTA = one (sequence, query head, 128-row Q tile).  16 warps in four warpgroups,
-// registers traded with setmaxnreg (128 x 40 + 128 x 88 + 256 x 192 = 512 x 128,
+// registers traded with setmaxnreg (128 x 56 + 128 x 88 + 256 x 184 = 512 x 128,
 // the launch allocation):
 //   WG0  warp 0: TMA producer (Q once, K / V tiles into rings)
 //        warp 1: TMEM owner and S issuer, warp 2: PV issuer (one thread each); warp 3 idle
-//          S(j)  = Q8 K8(j)^T   tcgen05.mma kind::i8 -> TMEM S buffer j % 2
+//          S(j)  = Q8 K8(j)^T   tcgen05.mma kind::i8 -> the TMEM S buffer
 //          PV(j) = P(j) V(j)    tcgen05.mma kind::f8f6f4 (e4m3) or kind::f16, A = P from
-//                               shared memory -> the PV block, a fresh FP32 accumulator
+//                               shared memory -> PV block j % 2, a fresh FP32 accumulator
 //   WG1  softmax of the even KV tiles, WG2 of the odd ones (one thread per query row,
 //        a whole 128-key row each); consecutive tiles pass the running max through
 //        shared memory, so the two warpgroups work on different tiles at once
 //   WG3  two-level accumulation O = alpha O + PV(j) held in TMEM, and the epilogue
 //
-// TMEM columns: S buffer 0 [0,128) (even tiles), S buffer 1 [128,256) (odd tiles),
-// the PV block [256, 256 + d) and the running O [384, 384 + d).  A softmax warpgroup
-// loads its S tile into registers and frees the buffer at once (P goes to shared
-// memory), so S(j + 2) can be computed while P(j) is being formed; the PV block and
-// the correction that folds it into O run behind, off the softmax's path.
+// TMEM columns: the S buffer [0,128), PV blocks 0 and 1 at [128, 128 + d) and
+// [256, 256 + d), the running O at [384, 384 + d).  A softmax warpgroup loads S(j) into
+// registers and frees the buffer at once (P goes to shared memory), so S(j + 1) is
+// computed while P(j) is being formed.  PV(j) lands in block j % 2 and the correction
+// warps fold it into O while PV(j + 1) runs in the other block.
 // Every S accumulates onto the magic pattern 0x4B400000 (fp32 1.5 * 2^23), so TMEM
 // returns bits(12582912 + S).  The pattern is written by the tensor core itself: before
 // the INT8 steps of S(j), one kind::f16 MMA with constant operands (every A entry 512,
@@ -41,11 +41,11 @@
 // own largest score, t = fma(S - S_max_c, c_c, nb_c) with c_c = q_scale k_scale_c sm_scale
 // log2 e and nb_c = S_max_c c_c - m' log2 e + log2 ps formed in fp64 and rounded once,
 // and 2^t is the hardware exponential (ex2.approx, within 2 ulp).  That p is within
-// about 15 fp32 ulps of the exact value whatever the logits' magnitude.  An e4m3 code
+// about 25 fp32 ulps of the exact value whatever the logits' magnitude.  An e4m3 code
 // is an integer decided by p, so for e4m3 P every p within 32 ulps of a rounding
-// midpoint is recomputed in fp64 from the definition and rounded from there: the codes
-// are those of the fp64 definition.  (A 16-bit P moves by one 16-bit ulp at such a
-// point; its codes are taken from the fast p.)
+// midpoint is decided again in fp64 from the definition (x - m against ln(mid / 448)):
+// the codes are those of the fp64 definition.  (A 16-bit P moves by one 16-bit ulp at
+// such a point; its codes are taken from the fast p.)
 #pragma once
 
 #include <type_traits>
@@ -57,9 +57,9 @@ namespace sage {
 
 constexpr int kAttnThreads = 512;
 constexpr int kAttnLaunchRegs = 128;  // 65536 / 512
-constexpr int kProducerRegs = 40;
+constexpr int kProducerRegs = 56;
 constexpr int kCorrectionRegs = 88;
-constexpr int kSoftmaxRegs = 192;
+constexpr int kSoftmaxRegs = 184;
 static_assert(128 * kProducerRegs + 128 * kCorrectionRegs + 256 * kSoftmaxRegs <=
                   kAttnThreads * kAttnLaunchRegs,
               "register split exceeds the launch allocation");
@@ -86,8 +86,9 @@ struct AttnArgs {
 
 template <int D, int PV>
 struct AttnCfg {
+  static constexpr bool kExact = PV == kPvE4m3;          // codes decided at midpoints
   static constexpr int kEB = PV == kPvE4m3 ? 1 : 2;      // bytes per P / V element
-  static constexpr int kKS = PV == kPvE4m3 ? 3 : 2;      // K ring stages
+  static constexpr int kKS = PV == kPvE4m3 ? 4 : 2;      // K ring stages (e4m3: one held by the helper)
   static constexpr int kVS = PV == kPvE4m3 ? 3 : 2;      // V ring stages
   static constexpr int kPBufs = PV == kPvE4m3 ? 3 : 2;   // P tiles in shared memory
   static constexpr int kTileQK = kBlkQ * D;              // bytes of one Q (or K) tile
@@ -97,21 +98,25 @@ struct AttnCfg {
   static constexpr int kKOff = kQOff + kTileQK;
   static constexpr int kVOff = kKOff + kKS * kTileQK;
   static constexpr int kPOff = kVOff + kVS * kTileV;
-  // constant f16 operands of the prefill MMA: 128 rows x 128 B each (128-byte swizzle
-  // atoms; every entry equal, so the layout is immaterial)
+  // constant f16 operands of the prefill MMA: 128 rows x 32 B each (32-byte swizzle atoms
+  // of 8 rows; every entry equal, so the layout is immaterial)
   static constexpr int kCAOff = kPOff + kPBufs * kTileP;
-  static constexpr int kCBOff = kCAOff + 128 * 128;
-  static constexpr int kMOff = kCBOff + 128 * 128;              // double mrun[2][128]
+  static constexpr int kCBOff = kCAOff + 128 * 32;
+  // exact e4m3 path, per P buffer: the softmax warps' flag ballots u32 [4 warps][4 chunks]
+  // and the rows' fp64 running max after the tile, double [128]
+  static constexpr int kFlagOff = kCBOff + 128 * 32;
+  static constexpr int kRowMOff = kFlagOff + (kExact ? kPBufs * 64 : 0);
+  static constexpr int kMOff = kRowMOff + (kExact ? kPBufs * 128 * 8 : 0);  // double mrun[2][128]
   static constexpr int kAOff = kMOff + 2 * 128 * 8;             // float alpha[4][128]
   static constexpr int kLOff = kAOff + kAlphaRing * 128 * 4;    // float lfin[2][128]
   static constexpr int kFOff = kLOff + 2 * 128 * 4;             // double mfin[2][128]
   static constexpr int kBarOff = kFOff + 2 * 128 * 8;
   // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS],
   // s_full[2], s_free[2], m_ready[2], p_full[PB], p_free[PB], a_full[4], a_free[4],
-  // pv_full, pv_free, epi, done
+  // pv_full[2], pv_free[2], epi, done, x_done[2], p_fixed[PB]
   static constexpr int kBarK = 1, kBarV = kBarK + 2 * kKS, kBarS = kBarV + 2 * kVS;
   static constexpr int kBarP = kBarS + 6, kBarA = kBarP + 2 * kPBufs, kBarX = kBarA + 2 * kAlphaRing;
-  static constexpr int kNumBars = kBarX + 4;
+  static constexpr int kNumBars = kBarX + 8 + kPBufs;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kSlotOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
@@ -178,7 +183,7 @@ __device__ __forceinline__ f2 pair_of(const uint32_t (&r)[32], int k) {
 constexpr uint32_t kMagicBits = 0x4B400000u;
 constexpr float kMagic = 12582912.0f;
 
-// max of 32 magic-offset scores (masked entries hold 0, below every valid value)
+// max of 32 magic-offset scores (masked entries hold -inf; 0 if the chunk has no valid one)
 __device__ __forceinline__ float max32(const uint32_t (&r)[32]) {
   float m0 = 0.0f, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
 #pragma unroll
@@ -212,100 +217,131 @@ __device__ __forceinline__ uint32_t cvt_pair(float lo, float hi) {
 // ---- exact e4m3 decision near a rounding midpoint
 // In the e4m3 normal range (p >= 2^-6) a code boundary is a value whose fp32 bits have
 // their low 20 bits equal to 0x80000 (the fp32 mantissa's first three bits are kept).
-// A fast p within kMidWin ulps of such a boundary is flagged: c = bits(p) + kMidWin has
-// (c & kMidMask) == 0x80000 exactly then.
+// A fast p within kMidWin ulps of such a boundary is flagged.  One integer multiply-add
+// tests it: key = bits(p) * 2^12 + 0x80020000 (mod 2^32) holds the low 20 bits of
+// bits(p) + 0x80020 in its top 20 bits, so key < 2^18 exactly when those low 20 bits
+// lie in [0x80000 - kMidWin, 0x80000 + kMidWin).  A chunk keeps the minimum key.
 constexpr uint32_t kMidWin = 32;
-constexpr uint32_t kMidMask = 0xFFFFFu & ~(2u * kMidWin - 1u);
-__device__ __forceinline__ uint32_t mid_flag(float p) {  // 0 iff p is flagged
-  return ((__float_as_uint(p) + kMidWin) & kMidMask) ^ 0x80000u;
+constexpr uint32_t kDetAdd = (0x80000u + kMidWin) << 12;
+constexpr uint32_t kDetLim = (2u * kMidWin) << 12;
+__device__ __forceinline__ uint32_t mid_key(float p) { return __float_as_uint(p) * 4096u + kDetAdd; }
+
+// ln((17 + 2k) / 16), k = 0..7: the log of the mantissa of the e4m3 rounding midpoint
+// 2^e (1 + (2k + 1) / 16) that lies between codes with mantissas 1 + k/8 and 1 + (k+1)/8
+__constant__ double kLnMidMant[8] = {
+    0.06062462181643484258, 0.17185025692665922234, 0.27193371548364175883,
+    0.36290549368936845314, 0.44628710262841951153, 0.52324814376454783652,
+    0.59470710774669278951, 0.66139848224536500826};
+constexpr double kLn2_64 = 0.69314718055994530942;
+constexpr double kLn448_64 = 6.10479323241498516161;
+
+// The value to convert for a flagged element.  The definition's p64 = 448 exp(x - m)
+// with x = ((S q_scale) k_scale) sm_scale lies above the midpoint `mid` exactly when
+// x - m > ln(mid / 448) = e ln 2 + ln(mantissa of mid) - ln 448, all in fp64.  The
+// returned float is on that side of the midpoint, one fp32 ulp away (or the midpoint
+// itself for an exact tie, which the conversion rounds to even, as the definition
+// does).  Below the e4m3 normal range, or at the saturation end, the fast p is kept.
+__device__ __forceinline__ float p_decided(float s, float sq, float sk, double scale, double m64,
+                                           float p) {
+  const uint32_t mb = ((__float_as_uint(p) + kMidWin) & 0xFFF00000u) | 0x80000u;
+  const float mid = __uint_as_float(mb);
+  if (!(mid >= 0x1p-6f) || mid > 448.0f) return p;
+  const double thr = static_cast<double>(static_cast<int>(mb >> 23) - 127) * kLn2_64 +
+                     (kLnMidMant[(mb >> 20) & 7u] - kLn448_64);
+  const double x = ((static_cast<double>(s) * static_cast<double>(sq)) * static_cast<double>(sk)) * scale;
+  const double dl = (x - m64) - thr;
+  return dl > 0.0 ? __uint_as_float(mb + 1u) : dl < 0.0 ? __uint_as_float(mb - 1u) : mid;
 }
 
-// The value to convert for a flagged element: the definition's p64 = 448 exp(x - m) with
-// x = ((S q_scale) k_scale) sm_scale in fp64, placed on the right side of the midpoint
-// next to the fast p (one fp32 ulp away, or the midpoint itself for an exact tie, which
-// the conversion then rounds to even, as the definition does).  Below the e4m3 normal
-// range, or at the saturation end, the fast p is kept.
-__device__ __noinline__ float p_at_midpoint(float s, float sq, float sk, double scale, double m64,
-                                            float p_fast) {
-  const uint32_t mid_bits = ((__float_as_uint(p_fast) + kMidWin) & 0xFFF00000u) | 0x80000u;
-  const float mid = __uint_as_float(mid_bits);
-  if (!(mid >= 0x1p-6f) || mid > 448.0f) return p_fast;
-  const double x = ((static_cast<double>(s) * static_cast<double>(sq)) * static_cast<double>(sk)) * scale;
-  const double p = 448.0 * exp(x - m64);
-  const double md = static_cast<double>(mid);
-  if (p > md) return __uint_as_float(mid_bits + 1u);
-  if (p < md) return __uint_as_float(mid_bits - 1u);
-  return mid;
+__device__ __forceinline__ uint32_t e4m3_code(float p) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(p));
+  return r & 0xFFu;
+}
+
+// Per-chunk constants of the fast p, formed from fp64 factors and rounded once:
+// c = q_scale k_scale sm_scale log2 e (at least the smallest normal float, so a dropped
+// key's -inf stays -inf) and nb = (S_max - 12582912) c - m' log2 e + log2 ps.  Every
+// operation is an explicit round-to-nearest one (no contraction), so the helper warp that
+// re-decides flagged codes forms the same two floats as the softmax.
+__device__ __forceinline__ double chunk_cc(double sq_sc, float sk) {
+  return __dmul_rn(__dmul_rn(sq_sc, static_cast<double>(sk)), kLog2E64);
+}
+__device__ __forceinline__ float chunk_ck(double cc) { return fmaxf(__double2float_rn(cc), 0x1p-126f); }
+__device__ __forceinline__ float chunk_nb(float hmax, double cc, double ml, double log2ps) {
+  return hmax > 1.0e6f
+      ? __double2float_rn(__dadd_rn(__dsub_rn(__dmul_rn(static_cast<double>(__fsub_rn(hmax, kMagic)), cc), ml), log2ps))
+      : 0.0f;
+}
+
+// Byte offset of 16-byte chunk k of row `row` in a K-major int8 tile of D-byte rows
+// written by TMA with the 128-byte (D = 128) or 64-byte (D = 64) swizzle.
+template <int D>
+__device__ __forceinline__ uint32_t swz_off(int row, int k) {
+  return D == 128 ? static_cast<uint32_t>(row * 128 + ((k ^ (row & 7)) << 4))
+                  : static_cast<uint32_t>(row * 64 + ((k ^ ((row >> 1) & 3)) << 4));
+}
+
+// Helper-warp work for one flagged (row r, chunk c) of a tile: lane i takes key 32c + i.
+// S is formed again from the int8 tiles (exact), then the softmax's own fp32 steps give
+// the same fast p; a p within kMidWin ulps of a midpoint is decided by p_decided and its
+// code byte rewritten in the row's slot of the P tile.
+template <int D>
+__device__ __forceinline__ void settle_chunk(uint32_t qbase, uint32_t kbase, uint32_t pbase, int r,
+                                             int c, int lane, bool drop, float sq, float sk,
+                                             double scale, double m64) {
+  const int key = 32 * c + lane;
+  int acc = 0;
+#pragma unroll
+  for (int k = 0; k < D / 16; ++k) {
+    uint32_t q4[4], k4[4];
+    ld_shared16(qbase + swz_off<D>(r, k), q4);
+    ld_shared16(kbase + swz_off<D>(key, k), k4);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc = __dp4a(static_cast<int>(q4[e]), static_cast<int>(k4[e]), acc);
+  }
+  const float sv = drop ? __uint_as_float(0xFF800000u) : kMagic + static_cast<float>(acc);
+  float hm = sv;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) hm = fmaxf(hm, __shfl_xor_sync(0xffffffffu, hm, o));
+  hm = fmaxf(hm, 0.0f);
+  const double cc = chunk_cc(__dmul_rn(static_cast<double>(sq), scale), sk);
+  const float nb = chunk_nb(hm, cc, __dmul_rn(m64, kLog2E64), kLog2_448_64);
+  const float p = ex2(__fmaf_rn(__fadd_rn(sv, -hm), chunk_ck(cc), nb));
+  if (mid_key(p) < kDetLim) {
+    const float pe = p_decided(__fsub_rn(sv, kMagic), sq, sk, scale, m64, p);
+    st_shared_u8(pbase + r * 128 + ((((2 * c + (lane >> 4)) ^ (r & 7)) & 7) << 4) + (lane & 15),
+                 e4m3_code(pe));
+  }
 }
 
 // P for the 32 keys of chunk c of one row: t = fma(S - S_max_c, ck, nb) (the difference
 // of two magic-offset floats is exact), p = 2^t, added into acc and written, in the PV
 // operand format, to the row's slot of a 128-byte-swizzled K-major P tile in shared
-// memory (`prow` = tile base + row * 128, `rx` = row % 8).  With kMasked, key i is kept
-// only when bit i of `keep` is set; dropped keys get p = 0.  With kExact (e4m3 P) codes
-// of p near a rounding midpoint are decided in fp64 by p_at_midpoint.
-struct ChunkExact {
-  float sq, sk;
-  double scale, m64;
-};
-
-// The 32 e4m3 codes of a chunk again, with every flagged p decided from the definition.
-// Rare (a flag hits about 6e-5 of the elements), so kept out of line: the chunk's scores
-// come in through local memory and the eight code words go back the same way.  The
-// fast p is recomputed with the same fp32 operations, so unflagged codes are unchanged.
-__device__ __noinline__ void e4m3_codes_exact(const uint32_t* s32, float hmax, float ck, float nb,
-                                             uint32_t keep, ChunkExact ex, uint32_t* w) {
-#pragma unroll 1
-  for (int i = 0; i < 32; i += 2) {
-    float p[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float sv = __uint_as_float(s32[i + e]);
-      p[e] = ((keep >> (i + e)) & 1u) ? ex2(__fmaf_rn(__fsub_rn(sv, hmax), ck, nb)) : 0.0f;
-      if (mid_flag(p[e]) == 0u) p[e] = p_at_midpoint(sv - kMagic, ex.sq, ex.sk, ex.scale, ex.m64, p[e]);
-    }
-    uint16_t two;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(two) : "f"(p[1]), "f"(p[0]));
-    if ((i >> 1) & 1) w[i >> 2] |= static_cast<uint32_t>(two) << 16;
-    else w[i >> 2] = two;
-  }
-}
-
-template <int PV, bool kMasked, bool kExact>
-__device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], float hmax, float ck, float nb,
-                                        f2& acc, uint32_t keep, uint32_t prow, int rx, int c,
-                                        const ChunkExact& ex) {
+// memory (`prow` = tile base + row * 128, `rx` = row % 8).  A dropped key holds S = -inf,
+// so its t is -inf and p = 0 (ck is at least the smallest normal float).  With kExact
+// (e4m3 P) the
+// chunk's smallest midpoint key is returned (below kDetLim: a p to decide again).
+template <int PV, bool kExact>
+__device__ __forceinline__ uint32_t p_chunk(const uint32_t (&r)[32], float hmax, float ck, float nb,
+                                            f2& acc, uint32_t prow, int rx, int c) {
   const f2 CK = f2_make(ck, ck), NB = f2_make(nb, nb), NH = f2_make(-hmax, -hmax);
   // one 16-byte chunk of the row at a time: 16 e4m3 codes or 8 16-bit values
   constexpr int kPerChunk = PV == kPvE4m3 ? 16 : 8;
   constexpr int kStores = 32 / kPerChunk;
   uint32_t w[kStores * 4];
-  uint32_t zmin = 0xFFFFFFFFu;
+  uint32_t kmin = 0xFFFFFFFFu;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const f2 t = f2_fma(f2_add(pair_of(r, i), NH), CK, NB);
     float p0 = ex2(t.x), p1 = ex2(t.y);
-    if (kMasked) {
-      p0 = ((keep >> (2 * i)) & 1u) ? p0 : 0.0f;
-      p1 = ((keep >> (2 * i + 1)) & 1u) ? p1 : 0.0f;
-    }
     acc = f2_add(acc, f2_make(p0, p1));
-    if constexpr (kExact) zmin = min(zmin, min(mid_flag(p0), mid_flag(p1)));
+    if constexpr (kExact) kmin = min(kmin, min(mid_key(p0), mid_key(p1)));
     const uint32_t two = cvt_pair<PV>(p0, p1);
     if constexpr (PV == kPvE4m3) {
       if (i & 1) w[i >> 1] |= two << 16; else w[i >> 1] = two;
     } else {
       w[i] = two;
-    }
-  }
-  if constexpr (kExact) {
-    if (__any_sync(0xffffffffu, zmin == 0u) && zmin == 0u) {
-      uint32_t s32[32], wx[8];  // local copies: w itself stays in registers
-#pragma unroll
-      for (int i = 0; i < 32; ++i) s32[i] = r[i];
-      e4m3_codes_exact(s32, hmax, ck, nb, kMasked ? keep : 0xFFFFFFFFu, ex, wx);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) w[i] = wx[i];
     }
   }
 #pragma unroll
@@ -322,6 +358,7 @@ __device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], float hmax, flo
                   w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
     }
   }
+  return kmin;
 }
 
 template <int D, class Seq, bool kFine, int PV>
@@ -332,14 +369,14 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ Seq seq, const __grid_constant__ AttnArgs a) {
   using L = AttnCfg<D, PV>;
   constexpr int KS = L::kKS, VS = L::kVS, PB = L::kPBufs;
-  constexpr bool kExact = PV == kPvE4m3;
+  constexpr bool kExact = L::kExact;
   constexpr uint32_t kSwizzle = (D == 128) ? 2u : 4u;  // UMMA layout type: 128B / 64B swizzle
   constexpr uint32_t kSboQK = 8u * D;                  // 8 rows of D bytes
   constexpr uint32_t kIdescS = idesc_i8(128, kKvTile);
   constexpr uint32_t kIdescPV = PV == kPvE4m3 ? idesc_e4m3_f32(128, D)
                                 : PV == kPvF16 ? idesc_f16_f32(128, D) : idesc_bf16_f32(128, D);
   constexpr uint32_t kIdescPre = idesc_f16_f32(128, kKvTile);
-  constexpr uint32_t kColPV = 256, kColO = 384;
+  constexpr uint32_t kColS = 0, kColPV = 128, kColO = 384;  // PV block b at kColPV + 128 b
   constexpr double kLog2Ps = PV == kPvE4m3 ? kLog2_448_64 : 0.0;
   constexpr float kLnPs = PV == kPvE4m3 ? kLn448 : 0.0f;
 
@@ -360,10 +397,14 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
   auto bar_pfree = [&](int b) { return bar0 + 8u * (L::kBarP + PB + b); };
   auto bar_afull = [&](int b) { return bar0 + 8u * (L::kBarA + b); };
   auto bar_afree = [&](int b) { return bar0 + 8u * (L::kBarA + kAlphaRing + b); };
-  const uint32_t bar_pvfull = bar0 + 8u * L::kBarX;
-  const uint32_t bar_pvfree = bar_pvfull + 8u;
-  const uint32_t bar_epi = bar_pvfull + 16u;
-  const uint32_t bar_done = bar_pvfull + 24u;
+  auto bar_pvfull = [&](int b) { return bar0 + 8u * (L::kBarX + b); };
+  auto bar_pvfree = [&](int b) { return bar0 + 8u * (L::kBarX + 2 + b); };
+  const uint32_t bar_epi = bar0 + 8u * (L::kBarX + 4);
+  const uint32_t bar_done = bar0 + 8u * (L::kBarX + 5);
+  auto bar_xdone = [&](int b) { return bar0 + 8u * (L::kBarX + 6 + b); };
+  auto bar_pfix = [&](int b) { return bar0 + 8u * (L::kBarX + 8 + b); };
+  uint32_t* fmask = reinterpret_cast<uint32_t*>(smem + L::kFlagOff);  // [buffer][warp][chunk]
+  double* rowm = reinterpret_cast<double*>(smem + L::kRowMOff);       // [buffer][row]
   double* mrun = reinterpret_cast<double*>(smem + L::kMOff);   // [tile % 2][row], fp64 max
   float* alph = reinterpret_cast<float*>(smem + L::kAOff);     // [tile % 4][row]
   float* lfin = reinterpret_cast<float*>(smem + L::kLOff);     // [wg][row]
@@ -407,23 +448,26 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < KS; ++s) { mbar_init(bar_kf(s), 1); mbar_init(bar_ke(s), 1); }
+    // a K stage is free once S has read it and (exact e4m3 P) the helper warp is done with it
+    for (int s = 0; s < KS; ++s) { mbar_init(bar_kf(s), 1); mbar_init(bar_ke(s), kExact ? 2 : 1); }
     for (int s = 0; s < VS; ++s) { mbar_init(bar_vf(s), 1); mbar_init(bar_ve(s), 1); }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar_sfull(s), 1);   // tcgen05.commit of S
-      mbar_init(bar_sfree(s), 4);   // the 4 softmax warps of the tile loaded S
+      mbar_init(bar_sfull(s), 1);   // tcgen05.commit of S(j), j % 2 == s
+      mbar_init(bar_sfree(s), 4);   // the 4 softmax warps of tile j loaded S(j)
       mbar_init(bar_mready(s), 4);  // the 4 softmax warps of the tile published its max
+      mbar_init(bar_pvfull(s), 1);  // tcgen05.commit of PV(j) into block j % 2
+      mbar_init(bar_pvfree(s), 4);  // the 4 correction warps read PV block s
+      mbar_init(bar_xdone(s), 4);   // the 4 softmax warps of tile j finished its exponentials
     }
     for (int s = 0; s < PB; ++s) {
       mbar_init(bar_pfull(s), 4);   // the 4 softmax warps wrote P
       mbar_init(bar_pfree(s), 1);   // tcgen05.commit of the PV that read it
+      mbar_init(bar_pfix(s), 1);    // the helper warp settled the tile's flagged codes
     }
     for (int s = 0; s < kAlphaRing; ++s) {
       mbar_init(bar_afull(s), 4);   // the 4 softmax warps wrote the tile's alpha
       mbar_init(bar_afree(s), 4);   // the 4 correction warps read it
     }
-    mbar_init(bar_pvfull, 1);       // tcgen05.commit of PV
-    mbar_init(bar_pvfree, 4);       // the 4 correction warps read the PV block
     mbar_init(bar_epi, 8);
     mbar_init(bar_done, 2);         // a commit from each MMA issuer
     fence_barrier_init();
@@ -441,7 +485,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     // prefill operands: f16 512.0 (0x6000) and 1536.0 (0x6600), two per word
     uint32_t* ca = reinterpret_cast<uint32_t*>(smem + L::kCAOff);
     uint32_t* cb = reinterpret_cast<uint32_t*>(smem + L::kCBOff);
-    for (int i = threadIdx.x; i < 128 * 128 / 4; i += kAttnThreads) {
+    for (int i = threadIdx.x; i < 128 * 32 / 4; i += kAttnThreads) {
       ca[i] = 0x60006000u;
       cb[i] = 0x66006600u;
     }
@@ -495,26 +539,26 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                global_timer_ns() - t0 < kWaitLimitNs) {}
     } else if ((warp == 1 || warp == 2) && lane == 0 && !dead) {
       // ========================================================== MMA issuers
-      // warp 1 issues every S(j), warp 2 every PV(j); each waits (suspended) only on its
-      // own inputs.  A thread's tcgen05.mma ops run in its issue order and its commits
-      // track its own ops, and the two streams share no operand: S(j) writes S buffer
-      // j % 2 from Q and K(j), PV(j) writes the PV block from P(j) and V(j).
+      // warp 1 issues every S(j), warp 2 every PV(j); each waits only on its own inputs.
+      // A thread's tcgen05.mma ops run in its issue order and its commits track its own
+      // ops, and the two streams share no operand: S(j) writes the S buffer from Q and
+      // K(j), PV(j) writes PV block j % 2 from P(j) and V(j).
       // descriptors differ only in their start-address field (bits 0-13, address >> 4)
       bool ok = mbar_wait<true>(bar_q, 0, 0x201);
       if (warp == 1) {
         const uint64_t dq = sdesc_kmajor(sbase + L::kQOff, kSboQK, kSwizzle);
         const uint64_t dk = sdesc_kmajor(sbase + L::kKOff, kSboQK, kSwizzle);
-        const uint64_t dca = sdesc_kmajor(sbase + L::kCAOff, 1024u, 2u);
-        const uint64_t dcb = sdesc_kmajor(sbase + L::kCBOff, 1024u, 2u);
+        const uint64_t dca = sdesc_kmajor(sbase + L::kCAOff, 256u, 6u);  // 32-byte swizzle
+        const uint64_t dcb = sdesc_kmajor(sbase + L::kCBOff, 256u, 6u);
         for (int js = 0; js < nkv && ok; ++js) {
-          // S(js) needs K(js) and its buffer free (tile js - 2 loaded by its softmax)
-          ok = (js < 2 || mbar_wait(bar_sfree(js & 1), ((js >> 1) - 1) & 1, 0x202)) &&
+          // S(js) needs K(js) and the S buffer free (S(js - 1) loaded by its softmax)
+          ok = (js == 0 || mbar_wait(bar_sfree((js - 1) & 1), ((js - 1) >> 1) & 1, 0x202)) &&
                mbar_wait(bar_kf(js % KS), (js / KS) & 1, 0x203);
           if (!ok) break;
           tc_fence_after();
           const int ks = js % KS;
           const uint64_t bk = dk + static_cast<uint64_t>((ks * L::kTileQK) >> 4);
-          const uint32_t d_tmem = tmem + 128u * (js & 1);
+          const uint32_t d_tmem = tmem + kColS;
           mma_f16_ss(d_tmem, dca, dcb, kIdescPre, 0u);  // every element := 12582912.0f
 #pragma unroll
           for (int s = 0; s < D / 32; ++s) mma_i8_ss(d_tmem, dq + 2u * s, bk + 2u * s, kIdescS, 1u);
@@ -525,17 +569,17 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const uint64_t dv = sdesc_kmajor(sbase + L::kVOff, 1024u, 2u);
         const uint64_t dp = sdesc_kmajor(sbase + L::kPOff, 1024u, 2u);
         for (int jp = 0; jp < nkv && ok; ++jp) {
-          // PV(jp) needs P(jp), V(jp) and the PV block free (tile jp - 1 read by the
+          // PV(jp) needs P(jp), V(jp) and PV block jp % 2 free (PV(jp - 2) read by the
           // correction)
-          ok = mbar_wait(bar_pfull(jp % PB), (jp / PB) & 1, 0x204) &&
+          ok = mbar_wait(kExact ? bar_pfix(jp % PB) : bar_pfull(jp % PB), (jp / PB) & 1, 0x204) &&
                mbar_wait(bar_vf(jp % VS), (jp / VS) & 1, 0x205) &&
-               (jp == 0 || mbar_wait(bar_pvfree, (jp - 1) & 1, 0x206));
+               (jp < 2 || mbar_wait(bar_pvfree(jp & 1), ((jp >> 1) - 1) & 1, 0x206));
           if (!ok) break;
           tc_fence_after();
           const int vs = jp % VS;
           const uint64_t bv = dv + static_cast<uint64_t>((vs * L::kTileV) >> 4);
           const uint64_t ap = dp + static_cast<uint64_t>(((jp % PB) * L::kTileP) >> 4);
-          const uint32_t d_tmem = tmem + kColPV;
+          const uint32_t d_tmem = tmem + kColPV + 128u * (jp & 1);
           if constexpr (PV == kPvE4m3) {
 #pragma unroll
             for (int s = 0; s < kKvTile / 32; ++s)  // 32 keys (32 bytes) per step
@@ -548,7 +592,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                          bv + ((blk * (D * 128) + w * 32) >> 4), kIdescPV, s > 0 ? 1u : 0u);
             }
           }
-          tc_commit(bar_pvfull);
+          tc_commit(bar_pvfull(jp & 1));
           tc_commit(bar_ve(vs));
           tc_commit(bar_pfree(jp % PB));
         }
@@ -557,16 +601,54 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       tc_commit(bar_done);
       const uint64_t t1 = global_timer_ns();
       while (!mbar_try_wait_sleep(bar_done, 0) && global_timer_ns() - t1 < kWaitLimitNs) {}
+    } else if (kExact && warp == 3 && !dead) {
+      // ========================================================== exact-decision helper
+      // After the softmax of tile j: every chunk a softmax warp flagged is settled by
+      // settle_chunk, then PV(j) may read P(j) (p_fixed) and the K stage may be refilled.
+      const uint32_t qbase = sbase + L::kQOff;
+      const float sq_tile = kFine ? 0.0f : a.q_scale[static_cast<int64_t>(hq) * (seq.t_pad / kBlkQ) + off / kBlkQ + qt];
+      constexpr int kblk = kFine ? kBlkKFine : kBlkK;
+      const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kblk) + off / kblk;
+      bool ok = true;
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int pb = j % PB, ks = j % KS;
+        ok = __all_sync(0xffffffffu, mbar_wait<true>(bar_pfull(pb), (j / PB) & 1, 0x501));
+        if (!ok) break;
+        const uint32_t kbase = sbase + L::kKOff + ks * L::kTileQK;
+        const uint32_t pbase = sbase + L::kPOff + pb * L::kTileP;
+        const int kv = j * kKvTile + lane;  // key of this lane in chunk 0
+        for (int w = 0; w < 4; ++w) {
+          for (int c = 0; c < 4; ++c) {
+            uint32_t bm = fmask[(pb * 4 + w) * 4 + c];
+            while (bm != 0u) {
+              const int r = 32 * w + (__ffs(bm) - 1);
+              bm &= bm - 1u;
+              const int grow = qt * kBlkQ + r;
+              const int key = kv + 32 * c;
+              const bool drop = key >= n || (a.causal && key > grow);
+              const float sq = kFine ? a.q_scale[static_cast<int64_t>(hq) * seq.t_pad + off + grow] : sq_tile;
+              const float sk = kFine ? ksc[4 * j + c] : ksc[2 * j + (c >> 1)];
+              settle_chunk<D>(qbase, kbase, pbase, r, c, lane, drop, sq, sk, a.scale, rowm[pb * 128 + r]);
+            }
+          }
+        }
+        fence_proxy_async_smem();  // rewritten codes -> visible to the tensor core
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar_pfix(pb));
+          mbar_arrive(bar_ke(ks));
+        }
+      }
     }
   } else if (wg <= 2) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     // ============================================================ softmax (every other tile)
-    const int h = wg - 1;           // tiles j with j % 2 == h, in S buffer h
+    const int h = wg - 1;           // tiles j with j % 2 == h
     const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const int grow = qt * kBlkQ + row;  // query index within the sequence
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_base + 128u * h;
+    const uint32_t tS = tmem + lane_base + kColS;
     const int rx = row & 7;
     bool ok = !dead;
     // this row's Q scale, and the K scales of the sequence; ksc32(j, c) is the scale of
@@ -577,14 +659,21 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     constexpr int kblk = kFine ? kBlkKFine : kBlkK;
     const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kblk) + off / kblk;
     auto ksc32 = [&](int j, int c) { return kFine ? ksc[4 * j + c] : ksc[2 * j + (c >> 1)]; };
-    const double sq_sc = static_cast<double>(sq) * a.scale;  // q_scale sm_scale
+    const double sq_sc = __dmul_rn(static_cast<double>(sq), a.scale);  // q_scale sm_scale
 
     float l = 0.0f;           // this warpgroup's partial sum, relative to mh
     double mh = -INFINITY;    // the max of this warpgroup's last tile
+    // K scales are fetched one tile of this warpgroup ahead, off the tile's critical path
+    float skn[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) skn[c] = h < nkv ? ksc32(h, c) : 0.0f;
     for (int j = h; j < nkv && ok; j += 2) {
       float sk[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) sk[c] = ksc32(j, c);
+      for (int c = 0; c < 4; ++c) {
+        sk[c] = skn[c];
+        skn[c] = j + 2 < nkv ? ksc32(j + 2, c) : 0.0f;
+      }
       const bool masked = (a.causal && j == qt) || (j + 1) * kKvTile > n;
       const int kv0 = j * kKvTile;  // first key of the tile
       auto dropped = [&](int key) { return key >= n || (a.causal && key > grow); };
@@ -599,19 +688,17 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       pin_regs(s[1]);
       pin_regs(s[2]);
       pin_regs(s[3]);
-      // S is in registers: the buffer may take S(j + 2)
+      // S is in registers: the buffer may take S(j + 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_sfree(h));
 
-      uint32_t keep[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
       if (masked) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          keep[c] = 0u;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            if (dropped(kv0 + 32 * c + i)) s[c][i] = 0u; else keep[c] |= 1u << i;
+            if (dropped(kv0 + 32 * c + i)) s[c][i] = 0xFF800000u;  // -inf
           }
         }
       }
@@ -657,18 +744,35 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
       // per chunk: c_c = q_scale k_scale_c sm_scale log2 e and
       // nb_c = S_max_c c_c - m' log2 e + log2 ps, in fp64, each rounded once
-      const double ml = m_new * kLog2E64;
+      const double ml = __dmul_rn(m_new, kLog2E64);
       const uint32_t prow = sbase + L::kPOff + (j % PB) * L::kTileP + row * 128;
+      // the two warpgroups take turns on the exponentials: tile j's start after tile
+      // j - 1's are done, so each runs alone on the MUFU pipe while the other one loads
+      // S, forms its maxima and waits on its barriers
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_xdone((j - 1) & 1), ((j - 1) >> 1) & 1, 0x309 + h));
+        if (!ok) break;
+      }
       f2 acc = make_float2(0.0f, 0.0f);
+      uint32_t kmin[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const double cc = sq_sc * static_cast<double>(sk[c]) * kLog2E64;
-        const float ck = static_cast<float>(cc);
-        const float nb = hm[c] > 1.0e6f
-            ? static_cast<float>(static_cast<double>(hm[c] - kMagic) * cc - ml + kLog2Ps) : 0.0f;
-        ChunkExact ex{sq, sk[c], a.scale, m_new};
-        if (masked) p_chunk<PV, true, kExact>(s[c], hm[c], ck, nb, acc, keep[c], prow, rx, c, ex);
-        else p_chunk<PV, false, kExact>(s[c], hm[c], ck, nb, acc, 0u, prow, rx, c, ex);
+        const double cc = chunk_cc(sq_sc, sk[c]);
+        kmin[c] = p_chunk<PV, kExact>(s[c], hm[c], chunk_ck(cc), chunk_nb(hm[c], cc, ml, kLog2Ps), acc,
+                                      prow, rx, c);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_xdone(j & 1));
+      if constexpr (kExact) {
+        // chunks holding a p near an e4m3 rounding midpoint (rare) go to the helper warp,
+        // which decides those codes from the definition before PV(j) is issued
+        const int pb = j % PB;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t bm = __ballot_sync(0xffffffffu, kmin[c] < kDetLim);
+          if (lane == 0) fmask[(pb * 4 + quarter) * 4 + c] = bm;
+        }
+        rowm[pb * 128 + row] = m_new;
       }
       l = l * ex2(static_cast<float>((mh - m_new) * kLog2E64)) + (acc.x + acc.y);
       mh = m_new;
@@ -688,20 +792,21 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const int row = quarter * 32 + lane;
     const int grow = qt * kBlkQ + row;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tPV = tmem + lane_base + kColPV;
+    const uint32_t tPV0 = tmem + lane_base + kColPV;
     const uint32_t tO = tmem + lane_base + kColO;
     bool ok = !dead;
 
     for (int j = 0; j < nkv && ok; ++j) {
       const int sa = j % kAlphaRing;
       ok = __all_sync(0xffffffffu, mbar_wait(bar_afull(sa), (j / kAlphaRing) & 1, 0x401)) &&
-           __all_sync(0xffffffffu, mbar_wait(bar_pvfull, j & 1, 0x402));
+           __all_sync(0xffffffffu, mbar_wait(bar_pvfull(j & 1), (j >> 1) & 1, 0x402));
       if (!ok) break;
       tc_fence_after();
       const float al = alph[sa * 128 + row];
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_afree(sa));
       const f2 AL = make_float2(al, al);
+      const uint32_t tPV = tPV0 + 128u * (j & 1);
       // O = alpha * O + PV_blk, 32 columns at a time (the first tile just copies PV_blk)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -714,10 +819,10 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         } else {
           tmem_wait_ld_tied(rp);
         }
-        if (c == D / 32 - 1) {  // the whole PV block has been read: PV(j + 1) may run
+        if (c == D / 32 - 1) {  // the whole PV block has been read: PV(j + 2) may run
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar_pvfree);
+          if (lane == 0) mbar_arrive(bar_pvfree(j & 1));
         }
         if (j > 0) {
 #pragma unroll
