@@ -88,7 +88,7 @@ template <int D, int PV>
 struct AttnCfg {
   static constexpr bool kExact = PV == kPvE4m3;          // codes decided at midpoints
   static constexpr int kEB = PV == kPvE4m3 ? 1 : 2;      // bytes per P / V element
-  static constexpr int kKS = PV == kPvE4m3 ? 4 : 2;      // K ring stages (e4m3: one held by the helper)
+  static constexpr int kKS = PV == kPvE4m3 ? 4 : 2;      // K ring stages (e4m3: K(j) is held until tile j is settled)
   static constexpr int kVS = PV == kPvE4m3 ? 3 : 2;      // V ring stages
   static constexpr int kPBufs = PV == kPvE4m3 ? 3 : 2;   // P tiles in shared memory
   static constexpr int kTileQK = kBlkQ * D;              // bytes of one Q (or K) tile
@@ -102,21 +102,17 @@ struct AttnCfg {
   // of 8 rows; every entry equal, so the layout is immaterial)
   static constexpr int kCAOff = kPOff + kPBufs * kTileP;
   static constexpr int kCBOff = kCAOff + 128 * 32;
-  // exact e4m3 path, per P buffer: the softmax warps' flag ballots u32 [4 warps][4 chunks]
-  // and the rows' fp64 running max after the tile, double [128]
-  static constexpr int kFlagOff = kCBOff + 128 * 32;
-  static constexpr int kRowMOff = kFlagOff + (kExact ? kPBufs * 64 : 0);
-  static constexpr int kMOff = kRowMOff + (kExact ? kPBufs * 128 * 8 : 0);  // double mrun[2][128]
+  static constexpr int kMOff = kCBOff + 128 * 32;               // double mrun[2][128]
   static constexpr int kAOff = kMOff + 2 * 128 * 8;             // float alpha[4][128]
   static constexpr int kLOff = kAOff + kAlphaRing * 128 * 4;    // float lfin[2][128]
   static constexpr int kFOff = kLOff + 2 * 128 * 4;             // double mfin[2][128]
   static constexpr int kBarOff = kFOff + 2 * 128 * 8;
   // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS],
   // s_full[2], s_free[2], m_ready[2], p_full[PB], p_free[PB], a_full[4], a_free[4],
-  // pv_full[2], pv_free[2], epi, done, x_done[2], p_fixed[PB]
+  // pv_full[2], pv_free[2], epi, done
   static constexpr int kBarK = 1, kBarV = kBarK + 2 * kKS, kBarS = kBarV + 2 * kVS;
   static constexpr int kBarP = kBarS + 6, kBarA = kBarP + 2 * kPBufs, kBarX = kBarA + 2 * kAlphaRing;
-  static constexpr int kNumBars = kBarX + 8 + kPBufs;
+  static constexpr int kNumBars = kBarX + 6;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kSlotOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
@@ -182,6 +178,15 @@ __device__ __forceinline__ f2 pair_of(const uint32_t (&r)[32], int k) {
 // are positive and ordered like S, and any difference of two is exact.
 constexpr uint32_t kMagicBits = 0x4B400000u;
 constexpr float kMagic = 12582912.0f;
+
+// a[i] for a small register array and a runtime index (a chain of selects)
+template <int N>
+__device__ __forceinline__ float pick(const float (&a)[N], int i) {
+  float v = a[0];
+#pragma unroll
+  for (int k = 1; k < N; ++k) v = i == k ? a[k] : v;
+  return v;
+}
 
 // max of 32 magic-offset scores (masked entries hold -inf; 0 if the chunk has no valid one)
 __device__ __forceinline__ float max32(const uint32_t (&r)[32]) {
@@ -259,18 +264,40 @@ __device__ __forceinline__ uint32_t e4m3_code(float p) {
   return r & 0xFFu;
 }
 
-// Per-chunk constants of the fast p, formed from fp64 factors and rounded once:
-// c = q_scale k_scale sm_scale log2 e (at least the smallest normal float, so a dropped
-// key's -inf stays -inf) and nb = (S_max - 12582912) c - m' log2 e + log2 ps.  Every
-// operation is an explicit round-to-nearest one (no contraction), so the helper warp that
-// re-decides flagged codes forms the same two floats as the softmax.
-__device__ __forceinline__ double chunk_cc(double sq_sc, float sk) {
-  return __dmul_rn(__dmul_rn(sq_sc, static_cast<double>(sk)), kLog2E64);
+// Exact conversions to fp64 that stay off the conversion unit (it shares its pipe with
+// the exponentials): an integer through the 2^52 + 2^31 magic, a non-negative float
+// through its bits (zero and subnormal values, rare, take the conversion instruction).
+__device__ __forceinline__ double int_to_f64(int v) {
+  return __dsub_rn(__hiloint2double(0x43300000, static_cast<int>(static_cast<uint32_t>(v) ^ 0x80000000u)),
+                   4503601774854144.0);
+}
+__device__ __forceinline__ double pos_f32_to_f64(float v) {
+  const uint32_t u = __float_as_uint(v);
+  if ((u >> 23) == 0u) {
+    double d;
+    asm volatile("cvt.f64.f32 %0, %1;" : "=d"(d) : "f"(v));
+    return d;
+  }
+  return __hiloint2double(static_cast<int>((((u >> 23) + 896u) << 20) | ((u & 0x7FFFFFu) >> 3)),
+                          static_cast<int>((u & 7u) << 29));
+}
+// S of a magic-offset score (exact: the float and the int differ by 0x4B400000 in bits)
+__device__ __forceinline__ int magic_to_int(float v) {
+  return static_cast<int>(__float_as_uint(v) - kMagicBits);
+}
+
+// Constants of the fast p for one K-scale block of a row, formed from fp64 factors and
+// rounded once: c = q_scale k_scale sm_scale log2 e (at least the smallest normal float,
+// so a dropped key's -inf stays -inf) and nb = S_max c - m' log2 e + log2 ps, S_max the
+// block's largest score.  Every operation is an explicit round-to-nearest one (no
+// contraction), so settle_chunk, which re-decides flagged codes, forms the same floats.
+__device__ __forceinline__ double chunk_cc(double sq_sc, double sk) {
+  return __dmul_rn(__dmul_rn(sq_sc, sk), kLog2E64);
 }
 __device__ __forceinline__ float chunk_ck(double cc) { return fmaxf(__double2float_rn(cc), 0x1p-126f); }
 __device__ __forceinline__ float chunk_nb(float hmax, double cc, double ml, double log2ps) {
   return hmax > 1.0e6f
-      ? __double2float_rn(__dadd_rn(__dsub_rn(__dmul_rn(static_cast<double>(__fsub_rn(hmax, kMagic)), cc), ml), log2ps))
+      ? __double2float_rn(__dadd_rn(__dsub_rn(__dmul_rn(int_to_f64(magic_to_int(hmax)), cc), ml), log2ps))
       : 0.0f;
 }
 
@@ -282,30 +309,40 @@ __device__ __forceinline__ uint32_t swz_off(int row, int k) {
                   : static_cast<uint32_t>(row * 64 + ((k ^ ((row >> 1) & 3)) << 4));
 }
 
-// Helper-warp work for one flagged (row r, chunk c) of a tile: lane i takes key 32c + i.
+// Settling of one flagged (row r, chunk c) of a tile by a whole warp: lane i takes key 32c + i.
 // S is formed again from the int8 tiles (exact), then the softmax's own fp32 steps give
 // the same fast p; a p within kMidWin ulps of a midpoint is decided by p_decided and its
 // code byte rewritten in the row's slot of the P tile.
+// Magic-offset score of query row r and key `key` of the tile from the int8 tiles
+// (-inf for a dropped key), exact.
 template <int D>
-__device__ __forceinline__ void settle_chunk(uint32_t qbase, uint32_t kbase, uint32_t pbase, int r,
-                                             int c, int lane, bool drop, float sq, float sk,
-                                             double scale, double m64) {
-  const int key = 32 * c + lane;
-  int acc = 0;
+__device__ __forceinline__ float score_at(uint32_t qbase, uint32_t kbase, int r, int key, bool drop) {
+  int acc[4] = {0, 0, 0, 0};  // four independent dot-product chains
 #pragma unroll
   for (int k = 0; k < D / 16; ++k) {
     uint32_t q4[4], k4[4];
     ld_shared16(qbase + swz_off<D>(r, k), q4);
     ld_shared16(kbase + swz_off<D>(key, k), k4);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc = __dp4a(static_cast<int>(q4[e]), static_cast<int>(k4[e]), acc);
+    for (int e = 0; e < 4; ++e) acc[e] = __dp4a(static_cast<int>(q4[e]), static_cast<int>(k4[e]), acc[e]);
   }
-  const float sv = drop ? __uint_as_float(0xFF800000u) : kMagic + static_cast<float>(acc);
+  const int sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  return drop ? __uint_as_float(0xFF800000u) : kMagic + static_cast<float>(sum);
+}
+
+// kCpb = chunks per K-scale block (2: 64-key blocks, 1: 32-key blocks); `drop_sib` says
+// whether this lane's key in the sibling chunk c ^ 1 is dropped.
+template <int D, int kCpb>
+__device__ __forceinline__ void settle_chunk(uint32_t qbase, uint32_t kbase, uint32_t pbase, int r,
+                                             int c, int lane, bool drop, bool drop_sib, float sq,
+                                             float sk, double scale, double m64) {
+  const float sv = score_at<D>(qbase, kbase, r, 32 * c + lane, drop);
   float hm = sv;
+  if (kCpb == 2) hm = fmaxf(hm, score_at<D>(qbase, kbase, r, 32 * (c ^ 1) + lane, drop_sib));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) hm = fmaxf(hm, __shfl_xor_sync(0xffffffffu, hm, o));
   hm = fmaxf(hm, 0.0f);
-  const double cc = chunk_cc(__dmul_rn(static_cast<double>(sq), scale), sk);
+  const double cc = chunk_cc(__dmul_rn(static_cast<double>(sq), scale), static_cast<double>(sk));
   const float nb = chunk_nb(hm, cc, __dmul_rn(m64, kLog2E64), kLog2_448_64);
   const float p = ex2(__fmaf_rn(__fadd_rn(sv, -hm), chunk_ck(cc), nb));
   if (mid_key(p) < kDetLim) {
@@ -401,10 +438,6 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
   auto bar_pvfree = [&](int b) { return bar0 + 8u * (L::kBarX + 2 + b); };
   const uint32_t bar_epi = bar0 + 8u * (L::kBarX + 4);
   const uint32_t bar_done = bar0 + 8u * (L::kBarX + 5);
-  auto bar_xdone = [&](int b) { return bar0 + 8u * (L::kBarX + 6 + b); };
-  auto bar_pfix = [&](int b) { return bar0 + 8u * (L::kBarX + 8 + b); };
-  uint32_t* fmask = reinterpret_cast<uint32_t*>(smem + L::kFlagOff);  // [buffer][warp][chunk]
-  double* rowm = reinterpret_cast<double*>(smem + L::kRowMOff);       // [buffer][row]
   double* mrun = reinterpret_cast<double*>(smem + L::kMOff);   // [tile % 2][row], fp64 max
   float* alph = reinterpret_cast<float*>(smem + L::kAOff);     // [tile % 4][row]
   float* lfin = reinterpret_cast<float*>(smem + L::kLOff);     // [wg][row]
@@ -448,8 +481,9 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    // a K stage is free once S has read it and (exact e4m3 P) the helper warp is done with it
-    for (int s = 0; s < KS; ++s) { mbar_init(bar_kf(s), 1); mbar_init(bar_ke(s), kExact ? 2 : 1); }
+    // a K stage is free once S has read it and (exact e4m3 P) the 4 softmax warps of the
+    // tile have settled their flagged chunks
+    for (int s = 0; s < KS; ++s) { mbar_init(bar_kf(s), 1); mbar_init(bar_ke(s), kExact ? 5 : 1); }
     for (int s = 0; s < VS; ++s) { mbar_init(bar_vf(s), 1); mbar_init(bar_ve(s), 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_sfull(s), 1);   // tcgen05.commit of S(j), j % 2 == s
@@ -457,12 +491,10 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       mbar_init(bar_mready(s), 4);  // the 4 softmax warps of the tile published its max
       mbar_init(bar_pvfull(s), 1);  // tcgen05.commit of PV(j) into block j % 2
       mbar_init(bar_pvfree(s), 4);  // the 4 correction warps read PV block s
-      mbar_init(bar_xdone(s), 4);   // the 4 softmax warps of tile j finished its exponentials
     }
     for (int s = 0; s < PB; ++s) {
       mbar_init(bar_pfull(s), 4);   // the 4 softmax warps wrote P
       mbar_init(bar_pfree(s), 1);   // tcgen05.commit of the PV that read it
-      mbar_init(bar_pfix(s), 1);    // the helper warp settled the tile's flagged codes
     }
     for (int s = 0; s < kAlphaRing; ++s) {
       mbar_init(bar_afull(s), 4);   // the 4 softmax warps wrote the tile's alpha
@@ -571,7 +603,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         for (int jp = 0; jp < nkv && ok; ++jp) {
           // PV(jp) needs P(jp), V(jp) and PV block jp % 2 free (PV(jp - 2) read by the
           // correction)
-          ok = mbar_wait(kExact ? bar_pfix(jp % PB) : bar_pfull(jp % PB), (jp / PB) & 1, 0x204) &&
+          ok = mbar_wait(bar_pfull(jp % PB), (jp / PB) & 1, 0x204) &&
                mbar_wait(bar_vf(jp % VS), (jp / VS) & 1, 0x205) &&
                (jp < 2 || mbar_wait(bar_pvfree(jp & 1), ((jp >> 1) - 1) & 1, 0x206));
           if (!ok) break;
@@ -601,44 +633,6 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       tc_commit(bar_done);
       const uint64_t t1 = global_timer_ns();
       while (!mbar_try_wait_sleep(bar_done, 0) && global_timer_ns() - t1 < kWaitLimitNs) {}
-    } else if (kExact && warp == 3 && !dead) {
-      // ========================================================== exact-decision helper
-      // After the softmax of tile j: every chunk a softmax warp flagged is settled by
-      // settle_chunk, then PV(j) may read P(j) (p_fixed) and the K stage may be refilled.
-      const uint32_t qbase = sbase + L::kQOff;
-      const float sq_tile = kFine ? 0.0f : a.q_scale[static_cast<int64_t>(hq) * (seq.t_pad / kBlkQ) + off / kBlkQ + qt];
-      constexpr int kblk = kFine ? kBlkKFine : kBlkK;
-      const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kblk) + off / kblk;
-      bool ok = true;
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int pb = j % PB, ks = j % KS;
-        ok = __all_sync(0xffffffffu, mbar_wait<true>(bar_pfull(pb), (j / PB) & 1, 0x501));
-        if (!ok) break;
-        const uint32_t kbase = sbase + L::kKOff + ks * L::kTileQK;
-        const uint32_t pbase = sbase + L::kPOff + pb * L::kTileP;
-        const int kv = j * kKvTile + lane;  // key of this lane in chunk 0
-        for (int w = 0; w < 4; ++w) {
-          for (int c = 0; c < 4; ++c) {
-            uint32_t bm = fmask[(pb * 4 + w) * 4 + c];
-            while (bm != 0u) {
-              const int r = 32 * w + (__ffs(bm) - 1);
-              bm &= bm - 1u;
-              const int grow = qt * kBlkQ + r;
-              const int key = kv + 32 * c;
-              const bool drop = key >= n || (a.causal && key > grow);
-              const float sq = kFine ? a.q_scale[static_cast<int64_t>(hq) * seq.t_pad + off + grow] : sq_tile;
-              const float sk = kFine ? ksc[4 * j + c] : ksc[2 * j + (c >> 1)];
-              settle_chunk<D>(qbase, kbase, pbase, r, c, lane, drop, sq, sk, a.scale, rowm[pb * 128 + r]);
-            }
-          }
-        }
-        fence_proxy_async_smem();  // rewritten codes -> visible to the tensor core
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(bar_pfix(pb));
-          mbar_arrive(bar_ke(ks));
-        }
-      }
     }
   } else if (wg <= 2) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
@@ -658,21 +652,24 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         : a.q_scale[static_cast<int64_t>(hq) * (seq.t_pad / kBlkQ) + off / kBlkQ + qt];
     constexpr int kblk = kFine ? kBlkKFine : kBlkK;
     const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kblk) + off / kblk;
-    auto ksc32 = [&](int j, int c) { return kFine ? ksc[4 * j + c] : ksc[2 * j + (c >> 1)]; };
-    const double sq_sc = __dmul_rn(static_cast<double>(sq), a.scale);  // q_scale sm_scale
+    // K-scale blocks per tile (64-key blocks, or 32-key ones with the per-thread option)
+    constexpr int kSB = kFine ? 4 : 2, kCpb = 4 / kSB;
+    auto kscb = [&](int j, int b) { return ksc[kSB * j + b]; };
+    const double sq_d = static_cast<double>(sq);
+    const double sq_sc = __dmul_rn(sq_d, a.scale);  // q_scale sm_scale
 
     float l = 0.0f;           // this warpgroup's partial sum, relative to mh
     double mh = -INFINITY;    // the max of this warpgroup's last tile
     // K scales are fetched one tile of this warpgroup ahead, off the tile's critical path
-    float skn[4];
+    float skn[kSB];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) skn[c] = h < nkv ? ksc32(h, c) : 0.0f;
+    for (int b = 0; b < kSB; ++b) skn[b] = h < nkv ? kscb(h, b) : 0.0f;
     for (int j = h; j < nkv && ok; j += 2) {
-      float sk[4];
+      float sk[kSB];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        sk[c] = skn[c];
-        skn[c] = j + 2 < nkv ? ksc32(j + 2, c) : 0.0f;
+      for (int b = 0; b < kSB; ++b) {
+        sk[b] = skn[b];
+        skn[b] = j + 2 < nkv ? kscb(j + 2, b) : 0.0f;
       }
       const bool masked = (a.causal && j == qt) || (j + 1) * kKvTile > n;
       const int kv0 = j * kKvTile;  // first key of the tile
@@ -702,16 +699,17 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
           }
         }
       }
-      // each chunk's largest score; the tile's max logit x = ((S q_scale) k_scale) sm_scale
-      // in fp64 (x is monotone in S within a chunk, so this is max_j x_j)
-      float hm[4];
+      // each K-scale block's largest score; the tile's max logit x = ((S q_scale) k_scale)
+      // sm_scale in fp64 (x is monotone in S within a block, so this is max_j x_j)
+      float hb[kSB];
+      double skd[kSB];
       double mt = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        hm[c] = max32(s[c]);
-        if (hm[c] > 1.0e6f) {
-          const double x = ((static_cast<double>(hm[c] - kMagic) * static_cast<double>(sq)) *
-                            static_cast<double>(sk[c])) * a.scale;
+      for (int b = 0; b < kSB; ++b) {
+        hb[b] = kCpb == 2 ? fmaxf(max32(s[2 * b]), max32(s[2 * b + 1])) : max32(s[b]);
+        skd[b] = pos_f32_to_f64(sk[b]);
+        if (hb[b] > 1.0e6f) {
+          const double x = __dmul_rn(__dmul_rn(__dmul_rn(int_to_f64(magic_to_int(hb[b])), sq_d), skd[b]), a.scale);
           mt = fmax(mt, x);
         }
       }
@@ -746,33 +744,50 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       // nb_c = S_max_c c_c - m' log2 e + log2 ps, in fp64, each rounded once
       const double ml = __dmul_rn(m_new, kLog2E64);
       const uint32_t prow = sbase + L::kPOff + (j % PB) * L::kTileP + row * 128;
-      // the two warpgroups take turns on the exponentials: tile j's start after tile
-      // j - 1's are done, so each runs alone on the MUFU pipe while the other one loads
-      // S, forms its maxima and waits on its barriers
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_xdone((j - 1) & 1), ((j - 1) >> 1) & 1, 0x309 + h));
-        if (!ok) break;
-      }
       f2 acc = make_float2(0.0f, 0.0f);
-      uint32_t kmin[4];
+      const int pb = j % PB;
+      float ckb[kSB], nbb[kSB];
+#pragma unroll
+      for (int b = 0; b < kSB; ++b) {
+        const double cc = chunk_cc(sq_sc, skd[b]);
+        ckb[b] = chunk_ck(cc);
+        nbb[b] = chunk_nb(hb[b], cc, ml, kLog2Ps);
+      }
+      uint32_t flag = 0u;  // lane c < 4: which rows of this warp have a flagged p in chunk c
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const double cc = chunk_cc(sq_sc, sk[c]);
-        kmin[c] = p_chunk<PV, kExact>(s[c], hm[c], chunk_ck(cc), chunk_nb(hm[c], cc, ml, kLog2Ps), acc,
-                                      prow, rx, c);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_xdone(j & 1));
-      if constexpr (kExact) {
-        // chunks holding a p near an e4m3 rounding midpoint (rare) go to the helper warp,
-        // which decides those codes from the definition before PV(j) is issued
-        const int pb = j % PB;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t bm = __ballot_sync(0xffffffffu, kmin[c] < kDetLim);
-          if (lane == 0) fmask[(pb * 4 + quarter) * 4 + c] = bm;
+        const uint32_t kmin = p_chunk<PV, kExact>(s[c], hb[c / kCpb], ckb[c / kCpb], nbb[c / kCpb], acc, prow, rx, c);
+        if constexpr (kExact) {
+          const uint32_t bm = __ballot_sync(0xffffffffu, kmin < kDetLim);
+          flag = lane == c ? bm : flag;
         }
-        rowm[pb * 128 + row] = m_new;
+      }
+      if constexpr (kExact) {
+        // Rare: chunks holding a p near an e4m3 rounding midpoint.  The warp settles them
+        // together (one key per lane, settle_chunk) before P(j) is published; then it
+        // releases K(j).
+        uint32_t nzc = __ballot_sync(0xffffffffu, lane < 4 && flag != 0u);
+        while (nzc != 0u) {
+          const int c = __ffs(nzc) - 1;
+          nzc &= nzc - 1u;
+          uint32_t bm = __shfl_sync(0xffffffffu, flag, c);
+          const float skc = pick(sk, c / kCpb);
+          const int key = j * kKvTile + 32 * c + lane, key2 = j * kKvTile + 32 * (c ^ 1) + lane;
+          while (bm != 0u) {
+            const int rl = __ffs(bm) - 1;
+            bm &= bm - 1u;
+            const int r = quarter * 32 + rl;
+            const int gr = qt * kBlkQ + r;
+            const double m64 = __shfl_sync(0xffffffffu, m_new, rl);
+            const float sqr = kFine ? __shfl_sync(0xffffffffu, sq, rl) : sq;
+            settle_chunk<D, kCpb>(sbase + L::kQOff, sbase + L::kKOff + (j % KS) * L::kTileQK,
+                                  sbase + L::kPOff + pb * L::kTileP, r, c, lane,
+                                  key >= n || (a.causal && key > gr), key2 >= n || (a.causal && key2 > gr),
+                                  sqr, skc, a.scale, m64);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_ke(j % KS));
       }
       l = l * ex2(static_cast<float>((mh - m_new) * kLog2E64)) + (acc.x + acc.y);
       mh = m_new;
