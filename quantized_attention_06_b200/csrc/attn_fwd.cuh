@@ -88,31 +88,30 @@ template <int D, int PV>
 struct AttnCfg {
   static constexpr bool kExact = PV == kPvE4m3;          // codes decided at midpoints
   static constexpr int kEB = PV == kPvE4m3 ? 1 : 2;      // bytes per P / V element
-  static constexpr int kKS = PV == kPvE4m3 ? 4 : 2;      // K ring stages (e4m3: K(j) is held until tile j is settled)
+  static constexpr int kKS = PV == kPvE4m3 ? 3 : 2;      // K ring stages
   static constexpr int kVS = PV == kPvE4m3 ? 3 : 2;      // V ring stages
-  static constexpr int kPBufs = PV == kPvE4m3 ? 3 : 2;   // P tiles in shared memory
+  static constexpr int kPBufs = PV == kPvE4m3 ? 2 : 1;   // P tiles in shared memory per Q tile
   static constexpr int kTileQK = kBlkQ * D;              // bytes of one Q (or K) tile
   static constexpr int kTileV = D * kKvTile * kEB;       // bytes of one V^T tile
   static constexpr int kTileP = kBlkQ * kKvTile * kEB;   // bytes of one P tile
-  static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kTileQK;
+  static constexpr int kQOff = 0;                        // Q tiles A and B
+  static constexpr int kKOff = kQOff + 2 * kTileQK;
   static constexpr int kVOff = kKOff + kKS * kTileQK;
-  static constexpr int kPOff = kVOff + kVS * kTileV;
+  static constexpr int kPOff = kVOff + kVS * kTileV;     // P tiles [Q tile][buffer]
   // constant f16 operands of the prefill MMA: 128 rows x 32 B each (32-byte swizzle atoms
   // of 8 rows; every entry equal, so the layout is immaterial)
-  static constexpr int kCAOff = kPOff + kPBufs * kTileP;
+  static constexpr int kCAOff = kPOff + 2 * kPBufs * kTileP;
   static constexpr int kCBOff = kCAOff + 128 * 32;
-  static constexpr int kMOff = kCBOff + 128 * 32;               // double mrun[2][128]
-  static constexpr int kAOff = kMOff + 2 * 128 * 8;             // float alpha[4][128]
-  static constexpr int kLOff = kAOff + kAlphaRing * 128 * 4;    // float lfin[2][128]
-  static constexpr int kFOff = kLOff + 2 * 128 * 4;             // double mfin[2][128]
+  static constexpr int kAOff = kCBOff + 128 * 32;                  // float alpha[2][4][128]
+  static constexpr int kLOff = kAOff + 2 * kAlphaRing * 128 * 4;   // float lfin[2][128]
+  static constexpr int kFOff = kLOff + 2 * 128 * 4;                // double mfin[2][128]
   static constexpr int kBarOff = kFOff + 2 * 128 * 8;
-  // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS],
-  // s_full[2], s_free[2], m_ready[2], p_full[PB], p_free[PB], a_full[4], a_free[4],
-  // pv_full[2], pv_free[2], epi, done
-  static constexpr int kBarK = 1, kBarV = kBarK + 2 * kKS, kBarS = kBarV + 2 * kVS;
-  static constexpr int kBarP = kBarS + 6, kBarA = kBarP + 2 * kPBufs, kBarX = kBarA + 2 * kAlphaRing;
-  static constexpr int kNumBars = kBarX + 6;
+  // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], then per Q tile:
+  // s_full, s_free, pv_done, o_ready, epi, p_full[PB], p_free[PB], a_full[4], a_free[4];
+  // and done
+  static constexpr int kBarK = 1, kBarV = kBarK + 2 * kKS, kBarX = kBarV + 2 * kVS;
+  static constexpr int kPerX = 5 + 2 * kPBufs + 2 * kAlphaRing;
+  static constexpr int kNumBars = kBarX + 2 * kPerX + 1;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kSlotOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
@@ -136,6 +135,11 @@ __device__ __forceinline__ f2 f2_fma(f2 a, f2 b, f2 c) {
 __device__ __forceinline__ f2 f2_add(f2 a, f2 b) {
   f2 d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(reinterpret_cast<uint64_t&>(d)) : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)));
+  return d;
+}
+__device__ __forceinline__ f2 f2_mul(f2 a, f2 b) {
+  f2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(reinterpret_cast<uint64_t&>(d)) : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)));
   return d;
 }
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -413,7 +417,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
   constexpr uint32_t kIdescPV = PV == kPvE4m3 ? idesc_e4m3_f32(128, D)
                                 : PV == kPvF16 ? idesc_f16_f32(128, D) : idesc_bf16_f32(128, D);
   constexpr uint32_t kIdescPre = idesc_f16_f32(128, kKvTile);
-  constexpr uint32_t kColS = 0, kColPV = 128, kColO = 384;  // PV block b at kColPV + 128 b
+  constexpr uint32_t kColO = 256;  // S of Q tile x at columns 128 x, its O at kColO + 128 x
   constexpr double kLog2Ps = PV == kPvE4m3 ? kLog2_448_64 : 0.0;
   constexpr float kLnPs = PV == kPvE4m3 ? kLn448 : 0.0f;
 
@@ -427,34 +431,34 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
   auto bar_ke = [&](int s) { return bar0 + 8u * (L::kBarK + KS + s); };
   auto bar_vf = [&](int s) { return bar0 + 8u * (L::kBarV + s); };
   auto bar_ve = [&](int s) { return bar0 + 8u * (L::kBarV + VS + s); };
-  auto bar_sfull = [&](int b) { return bar0 + 8u * (L::kBarS + b); };
-  auto bar_sfree = [&](int b) { return bar0 + 8u * (L::kBarS + 2 + b); };
-  auto bar_mready = [&](int b) { return bar0 + 8u * (L::kBarS + 4 + b); };
-  auto bar_pfull = [&](int b) { return bar0 + 8u * (L::kBarP + b); };
-  auto bar_pfree = [&](int b) { return bar0 + 8u * (L::kBarP + PB + b); };
-  auto bar_afull = [&](int b) { return bar0 + 8u * (L::kBarA + b); };
-  auto bar_afree = [&](int b) { return bar0 + 8u * (L::kBarA + kAlphaRing + b); };
-  auto bar_pvfull = [&](int b) { return bar0 + 8u * (L::kBarX + b); };
-  auto bar_pvfree = [&](int b) { return bar0 + 8u * (L::kBarX + 2 + b); };
-  const uint32_t bar_epi = bar0 + 8u * (L::kBarX + 4);
-  const uint32_t bar_done = bar0 + 8u * (L::kBarX + 5);
-  double* mrun = reinterpret_cast<double*>(smem + L::kMOff);   // [tile % 2][row], fp64 max
-  float* alph = reinterpret_cast<float*>(smem + L::kAOff);     // [tile % 4][row]
-  float* lfin = reinterpret_cast<float*>(smem + L::kLOff);     // [wg][row]
-  double* mfin = reinterpret_cast<double*>(smem + L::kFOff);   // [wg][row]
+  auto bx = [&](int x, int i) { return bar0 + 8u * (L::kBarX + x * L::kPerX + i); };
+  auto bar_sfull = [&](int x) { return bx(x, 0); };
+  auto bar_sfree = [&](int x) { return bx(x, 1); };
+  auto bar_pvdone = [&](int x) { return bx(x, 2); };
+  auto bar_oready = [&](int x) { return bx(x, 3); };
+  auto bar_epi = [&](int x) { return bx(x, 4); };
+  auto bar_pfull = [&](int x, int s) { return bx(x, 5 + s); };
+  auto bar_pfree = [&](int x, int s) { return bx(x, 5 + PB + s); };
+  auto bar_afull = [&](int x, int s) { return bx(x, 5 + 2 * PB + s); };
+  auto bar_afree = [&](int x, int s) { return bx(x, 5 + 2 * PB + kAlphaRing + s); };
+  const uint32_t bar_done = bar0 + 8u * (L::kBarX + 2 * L::kPerX);
+  float* alph = reinterpret_cast<float*>(smem + L::kAOff);     // [x][tile % 4][row]
+  float* lfin = reinterpret_cast<float*>(smem + L::kLOff);     // [x][row]
+  double* mfin = reinterpret_cast<double*>(smem + L::kFOff);   // [x][row]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wg = warp >> 2;
 
   // ---------------------------------------------------------------- work item
-  int b, hq, qt;
+  // CTA = (sequence, query head, pair of 128-row Q tiles 2 qp and 2 qp + 1)
+  int b, hq, qp;
   {
     int idx = blockIdx.x;
-    int ntiles;
+    int npair;
     if constexpr (std::is_same<Seq, SeqDense>::value) {
       b = 0;
-      ntiles = (seq_len(seq, 0) + kBlkQ - 1) / kBlkQ;
+      npair = ((seq_len(seq, 0) + kBlkQ - 1) / kBlkQ + 1) / 2;
     } else {
       int lo = 0, hi = seq.nseq - 1;
       while (lo < hi) {
@@ -464,44 +468,50 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       while (lo + 1 < seq.nseq && seq.cta[lo + 1] <= idx) ++lo;
       b = lo;
       idx -= seq.cta[b];
-      ntiles = (seq_len(seq, b) + kBlkQ - 1) / kBlkQ;
+      npair = ((seq_len(seq, b) + kBlkQ - 1) / kBlkQ + 1) / 2;
     }
     const int g = idx % a.group; idx /= a.group;
-    qt = idx % ntiles; idx /= ntiles;
+    qp = idx % npair; idx /= npair;
     const int hk = idx % a.hkv;
     if constexpr (std::is_same<Seq, SeqDense>::value) b = idx / a.hkv;
     hq = hk * a.group + g;
-    if (a.causal) qt = ntiles - 1 - qt;  // longest rows first
+    if (a.causal) qp = npair - 1 - qp;  // longest rows first
   }
   const int hk = hq / a.group;
   const int n = seq_len(seq, b);
   const int off = seq_off(seq, b);
-  const int nkv = a.causal ? qt + 1 : (n + kKvTile - 1) / kKvTile;
+  const bool hasB = 2 * qp + 1 < (n + kBlkQ - 1) / kBlkQ;  // the second Q tile exists
+  const int nX = hasB ? 2 : 1;
+  // KV tiles of the pair (causal: through the last Q tile's diagonal; Q tile A then sees
+  // one fully masked tile, whose P is zero)
+  const int nkv = a.causal ? 2 * qp + nX : (n + kKvTile - 1) / kKvTile;
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    // a K stage is free once S has read it and (exact e4m3 P) the 4 softmax warps of the
-    // tile have settled their flagged chunks
-    for (int s = 0; s < KS; ++s) { mbar_init(bar_kf(s), 1); mbar_init(bar_ke(s), kExact ? 5 : 1); }
-    for (int s = 0; s < VS; ++s) { mbar_init(bar_vf(s), 1); mbar_init(bar_ve(s), 1); }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar_sfull(s), 1);   // tcgen05.commit of S(j), j % 2 == s
-      mbar_init(bar_sfree(s), 4);   // the 4 softmax warps of tile j loaded S(j)
-      mbar_init(bar_mready(s), 4);  // the 4 softmax warps of the tile published its max
-      mbar_init(bar_pvfull(s), 1);  // tcgen05.commit of PV(j) into block j % 2
-      mbar_init(bar_pvfree(s), 4);  // the 4 correction warps read PV block s
+    // a K stage is free once S of both Q tiles read it and (exact e4m3 P) their softmax
+    // warps settled their flagged chunks; a V stage once both PV read it
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(bar_kf(s), 1);
+      mbar_init(bar_ke(s), nX + (kExact ? 4 * nX : 0));
     }
-    for (int s = 0; s < PB; ++s) {
-      mbar_init(bar_pfull(s), 4);   // the 4 softmax warps wrote P
-      mbar_init(bar_pfree(s), 1);   // tcgen05.commit of the PV that read it
+    for (int s = 0; s < VS; ++s) { mbar_init(bar_vf(s), 1); mbar_init(bar_ve(s), nX); }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar_sfull(x), 1);   // tcgen05.commit of S_x(j)
+      mbar_init(bar_sfree(x), 4);   // the 4 softmax warps of Q tile x loaded S_x(j)
+      mbar_init(bar_pvdone(x), 1);  // tcgen05.commit of PV_x(j) into O_x
+      mbar_init(bar_oready(x), 4);  // the 4 correction warps rescaled O_x for tile j
+      mbar_init(bar_epi(x), 4);     // the 4 softmax warps of Q tile x left l and m
+      for (int s = 0; s < PB; ++s) {
+        mbar_init(bar_pfull(x, s), 4);  // the 4 softmax warps wrote P_x
+        mbar_init(bar_pfree(x, s), 1);  // tcgen05.commit of the PV that read it
+      }
+      for (int s = 0; s < kAlphaRing; ++s) {
+        mbar_init(bar_afull(x, s), 4);  // the 4 softmax warps wrote the tile's alpha
+        mbar_init(bar_afree(x, s), 4);  // the 4 correction warps read it
+      }
     }
-    for (int s = 0; s < kAlphaRing; ++s) {
-      mbar_init(bar_afull(s), 4);   // the 4 softmax warps wrote the tile's alpha
-      mbar_init(bar_afree(s), 4);   // the 4 correction warps read it
-    }
-    mbar_init(bar_epi, 8);
-    mbar_init(bar_done, 2);         // a commit from each MMA issuer
+    mbar_init(bar_done, nX);        // a commit from each MMA issuer
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -534,8 +544,10 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     if (warp == 0 && lane == 0 && !dead) {
       // ========================================================== TMA producer
       bool ok = true;
-      mbar_arrive_expect_tx(bar_q, L::kTileQK);
-      tma_load_2d(sbase + L::kQOff, &tmap_q, 0, hq * seq.t_pad + off + qt * kBlkQ, bar_q);
+      mbar_arrive_expect_tx(bar_q, nX * L::kTileQK);
+      const int qrow = hq * seq.t_pad + off + 2 * qp * kBlkQ;
+      tma_load_2d(sbase + L::kQOff, &tmap_q, 0, qrow, bar_q);
+      if (hasB) tma_load_2d(sbase + L::kQOff + L::kTileQK, &tmap_q, 0, qrow + kBlkQ, bar_q);
       int nk = 0, nv = 0;  // loads issued
       for (int j = 0; j < nkv && ok; ++j) {
         const int ks = j % KS, vs = j % VS;
@@ -553,9 +565,9 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       bar_vf(vs));
         } else {
           // 16-bit V^T rows are 256 B per tile: two 128-byte-swizzled boxes of 64 keys
-          const int x = 2 * (off + j * kKvTile);
-          tma_load_2d(sbase + L::kVOff + vs * L::kTileV, &tmap_v, x, hk * D, bar_vf(vs));
-          tma_load_2d(sbase + L::kVOff + vs * L::kTileV + D * 128, &tmap_v, x + 128, hk * D,
+          const int xc = 2 * (off + j * kKvTile);
+          tma_load_2d(sbase + L::kVOff + vs * L::kTileV, &tmap_v, xc, hk * D, bar_vf(vs));
+          tma_load_2d(sbase + L::kVOff + vs * L::kTileV + D * 128, &tmap_v, xc + 128, hk * D,
                       bar_vf(vs));
         }
         ++nv;
@@ -569,65 +581,63 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
       for (int jj = max(0, nv - VS); jj < nv; ++jj)
         while (!mbar_try_wait_sleep(bar_vf(jj % VS), (jj / VS) & 1) &&
                global_timer_ns() - t0 < kWaitLimitNs) {}
-    } else if ((warp == 1 || warp == 2) && lane == 0 && !dead) {
+    } else if (warp >= 1 && warp <= nX && lane == 0 && !dead) {
       // ========================================================== MMA issuers
-      // warp 1 issues every S(j), warp 2 every PV(j); each waits only on its own inputs.
-      // A thread's tcgen05.mma ops run in its issue order and its commits track its own
-      // ops, and the two streams share no operand: S(j) writes the S buffer from Q and
-      // K(j), PV(j) writes PV block j % 2 from P(j) and V(j).
-      // descriptors differ only in their start-address field (bits 0-13, address >> 4)
+      // warp 1 issues every MMA of Q tile A, warp 2 every MMA of Q tile B.  Per KV tile j:
+      // S_x(j + 1) as soon as the softmax has S_x(j) in registers, then PV_x(j), which
+      // accumulates onto O_x once the correction warps have rescaled O_x for tile j.  A
+      // thread's tcgen05.mma ops run in its issue order and its commits track its own
+      // ops.  Descriptors differ only in their start-address field (address >> 4).
+      const int x = warp - 1;
       bool ok = mbar_wait<true>(bar_q, 0, 0x201);
-      if (warp == 1) {
-        const uint64_t dq = sdesc_kmajor(sbase + L::kQOff, kSboQK, kSwizzle);
-        const uint64_t dk = sdesc_kmajor(sbase + L::kKOff, kSboQK, kSwizzle);
-        const uint64_t dca = sdesc_kmajor(sbase + L::kCAOff, 256u, 6u);  // 32-byte swizzle
-        const uint64_t dcb = sdesc_kmajor(sbase + L::kCBOff, 256u, 6u);
-        for (int js = 0; js < nkv && ok; ++js) {
-          // S(js) needs K(js) and the S buffer free (S(js - 1) loaded by its softmax)
-          ok = (js == 0 || mbar_wait(bar_sfree((js - 1) & 1), ((js - 1) >> 1) & 1, 0x202)) &&
-               mbar_wait(bar_kf(js % KS), (js / KS) & 1, 0x203);
-          if (!ok) break;
-          tc_fence_after();
-          const int ks = js % KS;
-          const uint64_t bk = dk + static_cast<uint64_t>((ks * L::kTileQK) >> 4);
-          const uint32_t d_tmem = tmem + kColS;
-          mma_f16_ss(d_tmem, dca, dcb, kIdescPre, 0u);  // every element := 12582912.0f
+      const uint64_t dq = sdesc_kmajor(sbase + L::kQOff + x * L::kTileQK, kSboQK, kSwizzle);
+      const uint64_t dk = sdesc_kmajor(sbase + L::kKOff, kSboQK, kSwizzle);
+      const uint64_t dca = sdesc_kmajor(sbase + L::kCAOff, 256u, 6u);  // 32-byte swizzle
+      const uint64_t dcb = sdesc_kmajor(sbase + L::kCBOff, 256u, 6u);
+      const uint64_t dv = sdesc_kmajor(sbase + L::kVOff, 1024u, 2u);
+      const uint64_t dp = sdesc_kmajor(sbase + L::kPOff + x * PB * L::kTileP, 1024u, 2u);
+      const uint32_t tS = tmem + 128u * x, tO = tmem + kColO + 128u * x;
+      auto issue_s = [&](int js) {
+        if (!mbar_wait(bar_kf(js % KS), (js / KS) & 1, 0x203)) return false;
+        tc_fence_after();
+        const uint64_t bk = dk + static_cast<uint64_t>(((js % KS) * L::kTileQK) >> 4);
+        mma_f16_ss(tS, dca, dcb, kIdescPre, 0u);  // every element := 12582912.0f
 #pragma unroll
-          for (int s = 0; s < D / 32; ++s) mma_i8_ss(d_tmem, dq + 2u * s, bk + 2u * s, kIdescS, 1u);
-          tc_commit(bar_sfull(js & 1));
-          tc_commit(bar_ke(ks));
+        for (int s = 0; s < D / 32; ++s) mma_i8_ss(tS, dq + 2u * s, bk + 2u * s, kIdescS, 1u);
+        tc_commit(bar_sfull(x));
+        tc_commit(bar_ke(js % KS));
+        return true;
+      };
+      ok = ok && issue_s(0);
+      for (int jp = 0; jp < nkv && ok; ++jp) {
+        if (jp + 1 < nkv) {
+          ok = mbar_wait(bar_sfree(x), jp & 1, 0x202) && issue_s(jp + 1);
+          if (!ok) break;
         }
-      } else {
-        const uint64_t dv = sdesc_kmajor(sbase + L::kVOff, 1024u, 2u);
-        const uint64_t dp = sdesc_kmajor(sbase + L::kPOff, 1024u, 2u);
-        for (int jp = 0; jp < nkv && ok; ++jp) {
-          // PV(jp) needs P(jp), V(jp) and PV block jp % 2 free (PV(jp - 2) read by the
-          // correction)
-          ok = mbar_wait(bar_pfull(jp % PB), (jp / PB) & 1, 0x204) &&
-               mbar_wait(bar_vf(jp % VS), (jp / VS) & 1, 0x205) &&
-               (jp < 2 || mbar_wait(bar_pvfree(jp & 1), ((jp >> 1) - 1) & 1, 0x206));
-          if (!ok) break;
-          tc_fence_after();
-          const int vs = jp % VS;
-          const uint64_t bv = dv + static_cast<uint64_t>((vs * L::kTileV) >> 4);
-          const uint64_t ap = dp + static_cast<uint64_t>(((jp % PB) * L::kTileP) >> 4);
-          const uint32_t d_tmem = tmem + kColPV + 128u * (jp & 1);
-          if constexpr (PV == kPvE4m3) {
+        // PV(jp) needs P(jp), V(jp) and, after the first tile, O rescaled for tile jp
+        ok = mbar_wait(bar_pfull(x, jp % PB), (jp / PB) & 1, 0x204) &&
+             mbar_wait(bar_vf(jp % VS), (jp / VS) & 1, 0x205) &&
+             (jp == 0 || mbar_wait(bar_oready(x), (jp - 1) & 1, 0x206));
+        if (!ok) break;
+        tc_fence_after();
+        const int vs = jp % VS;
+        const uint64_t bv = dv + static_cast<uint64_t>((vs * L::kTileV) >> 4);
+        const uint64_t ap = dp + static_cast<uint64_t>(((jp % PB) * L::kTileP) >> 4);
+        if constexpr (PV == kPvE4m3) {
 #pragma unroll
-            for (int s = 0; s < kKvTile / 32; ++s)  // 32 keys (32 bytes) per step
-              mma_f8_ss(d_tmem, ap + 2u * s, bv + 2u * s, kIdescPV, s > 0 ? 1u : 0u);
-          } else {
+          for (int s = 0; s < kKvTile / 32; ++s)  // 32 keys (32 bytes) per step
+            mma_f8_ss(tO, ap + 2u * s, bv + 2u * s, kIdescPV, (jp > 0 || s > 0) ? 1u : 0u);
+        } else {
 #pragma unroll
-            for (int s = 0; s < kKvTile / 16; ++s) {  // 16 keys (32 bytes) per step
-              const uint32_t blk = s >> 2, w = s & 3;  // 64-key swizzle block, step within it
-              mma_f16_ss(d_tmem, ap + ((blk * (kBlkQ * 128) + w * 32) >> 4),
-                         bv + ((blk * (D * 128) + w * 32) >> 4), kIdescPV, s > 0 ? 1u : 0u);
-            }
+          for (int s = 0; s < kKvTile / 16; ++s) {  // 16 keys (32 bytes) per step
+            const uint32_t blk = s >> 2, w = s & 3;  // 64-key swizzle block, step within it
+            mma_f16_ss(tO, ap + ((blk * (kBlkQ * 128) + w * 32) >> 4),
+                       bv + ((blk * (D * 128) + w * 32) >> 4), kIdescPV, (jp > 0 || s > 0) ? 1u : 0u);
           }
-          tc_commit(bar_pvfull(jp & 1));
-          tc_commit(bar_ve(vs));
-          tc_commit(bar_pfree(jp % PB));
         }
+        tc_commit(bar_pvdone(x));
+        tc_commit(bar_ve(vs));
+        tc_commit(bar_pfree(x, jp % PB));
       }
       // every MMA issued by this thread has completed before TMEM is released
       tc_commit(bar_done);
@@ -636,236 +646,223 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     }
   } else if (wg <= 2) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-    // ============================================================ softmax (every other tile)
-    const int h = wg - 1;           // tiles j with j % 2 == h
-    const int quarter = warp & 3;   // TMEM lane quarter this warp may access
-    const int row = quarter * 32 + lane;
-    const int grow = qt * kBlkQ + row;  // query index within the sequence
-    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_base + kColS;
-    const int rx = row & 7;
-    bool ok = !dead;
-    // this row's Q scale, and the K scales of the sequence; ksc32(j, c) is the scale of
-    // keys 32c .. 32c + 31 of KV tile j (its 64-token block, or its own 32-token block)
-    const float sq = kFine
-        ? a.q_scale[static_cast<int64_t>(hq) * seq.t_pad + off + qt * kBlkQ + row]
-        : a.q_scale[static_cast<int64_t>(hq) * (seq.t_pad / kBlkQ) + off / kBlkQ + qt];
-    constexpr int kblk = kFine ? kBlkKFine : kBlkK;
-    const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kblk) + off / kblk;
-    // K-scale blocks per tile (64-key blocks, or 32-key ones with the per-thread option)
-    constexpr int kSB = kFine ? 4 : 2, kCpb = 4 / kSB;
-    auto kscb = [&](int j, int b) { return ksc[kSB * j + b]; };
-    const double sq_d = static_cast<double>(sq);
-    const double sq_sc = __dmul_rn(sq_d, a.scale);  // q_scale sm_scale
+    // ============================================================ softmax of Q tile x
+    const int x = wg - 1;
+    if (x < nX) {
+      const int qt = 2 * qp + x;
+      const int quarter = warp & 3;   // TMEM lane quarter this warp may access
+      const int row = quarter * 32 + lane;
+      const int grow = qt * kBlkQ + row;  // query index within the sequence
+      const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+      const uint32_t tS = tmem + lane_base + 128u * x;
+      const int rx = row & 7;
+      bool ok = !dead;
+      // this row's Q scale, and the K scales of the sequence
+      const float sq = kFine
+          ? a.q_scale[static_cast<int64_t>(hq) * seq.t_pad + off + qt * kBlkQ + row]
+          : a.q_scale[static_cast<int64_t>(hq) * (seq.t_pad / kBlkQ) + off / kBlkQ + qt];
+      constexpr int kblk = kFine ? kBlkKFine : kBlkK;
+      const float* ksc = a.k_scale + static_cast<int64_t>(hk) * (seq.t_pad / kblk) + off / kblk;
+      // K-scale blocks per tile (64-key blocks, or 32-key ones with the per-thread option)
+      constexpr int kSB = kFine ? 4 : 2, kCpb = 4 / kSB;
+      auto kscb = [&](int j, int bb) { return ksc[kSB * j + bb]; };
+      const double sq_d = static_cast<double>(sq);
+      const double sq_sc = __dmul_rn(sq_d, a.scale);  // q_scale sm_scale
 
-    float l = 0.0f;           // this warpgroup's partial sum, relative to mh
-    double mh = -INFINITY;    // the max of this warpgroup's last tile
-    // K scales are fetched one tile of this warpgroup ahead, off the tile's critical path
-    float skn[kSB];
+      // K scales are fetched one tile ahead, off the tile's critical path
+      float skn[kSB];
 #pragma unroll
-    for (int b = 0; b < kSB; ++b) skn[b] = h < nkv ? kscb(h, b) : 0.0f;
-    for (int j = h; j < nkv && ok; j += 2) {
-      float sk[kSB];
+      for (int bb = 0; bb < kSB; ++bb) skn[bb] = kscb(0, bb);
+      float l = 0.0f;            // running sum, relative to m_run
+      double m_run = -INFINITY;  // running max of the logits (fp64, as the definition)
+      for (int j = 0; j < nkv && ok; ++j) {
+        float sk[kSB];
 #pragma unroll
-      for (int b = 0; b < kSB; ++b) {
-        sk[b] = skn[b];
-        skn[b] = j + 2 < nkv ? kscb(j + 2, b) : 0.0f;
-      }
-      const bool masked = (a.causal && j == qt) || (j + 1) * kKvTile > n;
-      const int kv0 = j * kKvTile;  // first key of the tile
-      auto dropped = [&](int key) { return key >= n || (a.causal && key > grow); };
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull(h), (j >> 1) & 1, 0x301 + h));
-      if (!ok) break;
-      tc_fence_after();
+        for (int bb = 0; bb < kSB; ++bb) {
+          sk[bb] = skn[bb];
+          skn[bb] = j + 1 < nkv ? kscb(j + 1, bb) : 0.0f;
+        }
+        const bool masked = (a.causal && j >= qt) || (j + 1) * kKvTile > n;
+        const int kv0 = j * kKvTile;  // first key of the tile
+        auto dropped = [&](int key) { return key >= n || (a.causal && key > grow); };
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull(x), j & 1, 0x301 + x));
+        if (!ok) break;
+        tc_fence_after();
 
-      uint32_t s[4][32];
+        uint32_t s[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32u * c, s[c]);
-      tmem_wait_ld_tied(s[0]);
-      pin_regs(s[1]);
-      pin_regs(s[2]);
-      pin_regs(s[3]);
-      // S is in registers: the buffer may take S(j + 1)
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_sfree(h));
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32u * c, s[c]);
+        tmem_wait_ld_tied(s[0]);
+        pin_regs(s[1]);
+        pin_regs(s[2]);
+        pin_regs(s[3]);
+        // S is in registers: the buffer may take S(j + 1)
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_sfree(x));
 
-      if (masked) {
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (dropped(kv0 + 32 * c + i)) s[c][i] = 0xFF800000u;  // -inf
+            }
+          }
+        }
+        // each K-scale block's largest score; the tile's max logit x = ((S q_scale) k_scale)
+        // sm_scale in fp64 (x is monotone in S within a block, so this is max_j x_j)
+        float hb[kSB];
+        double skd[kSB];
+        double mt = -INFINITY;
+#pragma unroll
+        for (int bb = 0; bb < kSB; ++bb) {
+          hb[bb] = kCpb == 2 ? fmaxf(max32(s[2 * bb]), max32(s[2 * bb + 1])) : max32(s[bb]);
+          skd[bb] = pos_f32_to_f64(sk[bb]);
+          if (hb[bb] > 1.0e6f) {
+            const double xm = __dmul_rn(__dmul_rn(__dmul_rn(int_to_f64(magic_to_int(hb[bb])), sq_d), skd[bb]), a.scale);
+            mt = fmax(mt, xm);
+          }
+        }
+        const double m_new = fmax(m_run, mt);
+        // alpha = e^(m - m') rescales l here and O in the correction warps (slot j % 4)
+        const float alpha = ex2(static_cast<float>((m_run - m_new) * kLog2E64));
+        if (j >= kAlphaRing) {
+          const int jo = j - kAlphaRing;
+          ok = __all_sync(0xffffffffu, mbar_wait(bar_afree(x, jo % kAlphaRing), (jo / kAlphaRing) & 1, 0x305 + x));
+          if (!ok) break;
+        }
+        alph[(x * kAlphaRing + j % kAlphaRing) * 128 + row] = alpha;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_afull(x, j % kAlphaRing));
+        // the P buffer of tile j was last read by PV(j - PB)
+        const int pb = j % PB;
+        if (j >= PB) {
+          const int jo = j - PB;
+          ok = __all_sync(0xffffffffu, mbar_wait(bar_pfree(x, jo % PB), (jo / PB) & 1, 0x307 + x));
+          if (!ok) break;
+        }
+
+        // per K-scale block: c = q_scale k_scale sm_scale log2 e and
+        // nb = S_max c - m' log2 e + log2 ps, in fp64, each rounded once
+        const double ml = __dmul_rn(m_new, kLog2E64);
+        const uint32_t ptile = sbase + L::kPOff + (x * PB + pb) * L::kTileP;
+        const uint32_t prow = ptile + row * 128;
+        f2 acc = make_float2(0.0f, 0.0f);
+        float ckb[kSB], nbb[kSB];
+#pragma unroll
+        for (int bb = 0; bb < kSB; ++bb) {
+          const double cc = chunk_cc(sq_sc, skd[bb]);
+          ckb[bb] = chunk_ck(cc);
+          nbb[bb] = chunk_nb(hb[bb], cc, ml, kLog2Ps);
+        }
+        uint32_t flag = 0u;  // lane c < 4: which rows of this warp have a flagged p in chunk c
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (dropped(kv0 + 32 * c + i)) s[c][i] = 0xFF800000u;  // -inf
+          const uint32_t kmin = p_chunk<PV, kExact>(s[c], hb[c / kCpb], ckb[c / kCpb], nbb[c / kCpb], acc, prow, rx, c);
+          if constexpr (kExact) {
+            const uint32_t bm = __ballot_sync(0xffffffffu, kmin < kDetLim);
+            flag = lane == c ? bm : flag;
           }
         }
-      }
-      // each K-scale block's largest score; the tile's max logit x = ((S q_scale) k_scale)
-      // sm_scale in fp64 (x is monotone in S within a block, so this is max_j x_j)
-      float hb[kSB];
-      double skd[kSB];
-      double mt = -INFINITY;
-#pragma unroll
-      for (int b = 0; b < kSB; ++b) {
-        hb[b] = kCpb == 2 ? fmaxf(max32(s[2 * b]), max32(s[2 * b + 1])) : max32(s[b]);
-        skd[b] = pos_f32_to_f64(sk[b]);
-        if (hb[b] > 1.0e6f) {
-          const double x = __dmul_rn(__dmul_rn(__dmul_rn(int_to_f64(magic_to_int(hb[b])), sq_d), skd[b]), a.scale);
-          mt = fmax(mt, x);
-        }
-      }
-      // the running max after the previous tile comes from the other warpgroup
-      double m_prev = -INFINITY;
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_mready((j - 1) & 1), ((j - 1) >> 1) & 1, 0x303 + h));
-        if (!ok) break;
-        m_prev = mrun[((j - 1) & 1) * 128 + row];
-      }
-      const double m_new = fmax(m_prev, mt);
-      mrun[(j & 1) * 128 + row] = m_new;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_mready(j & 1));
-      // alpha = e^(m - m') for the correction warps (slot j % 4)
-      if (j >= kAlphaRing) {
-        const int jo = j - kAlphaRing;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_afree(jo % kAlphaRing), (jo / kAlphaRing) & 1, 0x305 + h));
-        if (!ok) break;
-      }
-      alph[(j % kAlphaRing) * 128 + row] = ex2(static_cast<float>((m_prev - m_new) * kLog2E64));
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_afull(j % kAlphaRing));
-      // the P buffer of tile j was last read by PV(j - PB)
-      if (j >= PB) {
-        const int jo = j - PB;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_pfree(jo % PB), (jo / PB) & 1, 0x307 + h));
-        if (!ok) break;
-      }
-
-      // per chunk: c_c = q_scale k_scale_c sm_scale log2 e and
-      // nb_c = S_max_c c_c - m' log2 e + log2 ps, in fp64, each rounded once
-      const double ml = __dmul_rn(m_new, kLog2E64);
-      const uint32_t prow = sbase + L::kPOff + (j % PB) * L::kTileP + row * 128;
-      f2 acc = make_float2(0.0f, 0.0f);
-      const int pb = j % PB;
-      float ckb[kSB], nbb[kSB];
-#pragma unroll
-      for (int b = 0; b < kSB; ++b) {
-        const double cc = chunk_cc(sq_sc, skd[b]);
-        ckb[b] = chunk_ck(cc);
-        nbb[b] = chunk_nb(hb[b], cc, ml, kLog2Ps);
-      }
-      uint32_t flag = 0u;  // lane c < 4: which rows of this warp have a flagged p in chunk c
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint32_t kmin = p_chunk<PV, kExact>(s[c], hb[c / kCpb], ckb[c / kCpb], nbb[c / kCpb], acc, prow, rx, c);
         if constexpr (kExact) {
-          const uint32_t bm = __ballot_sync(0xffffffffu, kmin < kDetLim);
-          flag = lane == c ? bm : flag;
-        }
-      }
-      if constexpr (kExact) {
-        // Rare: chunks holding a p near an e4m3 rounding midpoint.  The warp settles them
-        // together (one key per lane, settle_chunk) before P(j) is published; then it
-        // releases K(j).
-        uint32_t nzc = __ballot_sync(0xffffffffu, lane < 4 && flag != 0u);
-        while (nzc != 0u) {
-          const int c = __ffs(nzc) - 1;
-          nzc &= nzc - 1u;
-          uint32_t bm = __shfl_sync(0xffffffffu, flag, c);
-          const float skc = pick(sk, c / kCpb);
-          const int key = j * kKvTile + 32 * c + lane, key2 = j * kKvTile + 32 * (c ^ 1) + lane;
-          while (bm != 0u) {
-            const int rl = __ffs(bm) - 1;
-            bm &= bm - 1u;
-            const int r = quarter * 32 + rl;
-            const int gr = qt * kBlkQ + r;
-            const double m64 = __shfl_sync(0xffffffffu, m_new, rl);
-            const float sqr = kFine ? __shfl_sync(0xffffffffu, sq, rl) : sq;
-            settle_chunk<D, kCpb>(sbase + L::kQOff, sbase + L::kKOff + (j % KS) * L::kTileQK,
-                                  sbase + L::kPOff + pb * L::kTileP, r, c, lane,
-                                  key >= n || (a.causal && key > gr), key2 >= n || (a.causal && key2 > gr),
-                                  sqr, skc, a.scale, m64);
+          // Rare: chunks holding a p near an e4m3 rounding midpoint.  The warp settles them
+          // together (one key per lane, settle_chunk) before P(j) is published; then it
+          // releases K(j).
+          uint32_t nzc = __ballot_sync(0xffffffffu, lane < 4 && flag != 0u);
+          while (nzc != 0u) {
+            const int c = __ffs(nzc) - 1;
+            nzc &= nzc - 1u;
+            uint32_t bm = __shfl_sync(0xffffffffu, flag, c);
+            const float skc = pick(sk, c / kCpb);
+            const int key = kv0 + 32 * c + lane, key2 = kv0 + 32 * (c ^ 1) + lane;
+            while (bm != 0u) {
+              const int rl = __ffs(bm) - 1;
+              bm &= bm - 1u;
+              const int r = quarter * 32 + rl;
+              const int gr = qt * kBlkQ + r;
+              const double m64 = __shfl_sync(0xffffffffu, m_new, rl);
+              const float sqr = kFine ? __shfl_sync(0xffffffffu, sq, rl) : sq;
+              settle_chunk<D, kCpb>(sbase + L::kQOff + x * L::kTileQK,
+                                    sbase + L::kKOff + (j % KS) * L::kTileQK, ptile, r, c, lane,
+                                    key >= n || (a.causal && key > gr), key2 >= n || (a.causal && key2 > gr),
+                                    sqr, skc, a.scale, m64);
+            }
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_ke(j % KS));
         }
+        l = l * alpha + (acc.x + acc.y);
+        m_run = m_new;
+        fence_proxy_async_smem();  // P stores -> visible to the tensor core
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_ke(j % KS));
+        if (lane == 0) mbar_arrive(bar_pfull(x, pb));
       }
-      l = l * ex2(static_cast<float>((mh - m_new) * kLog2E64)) + (acc.x + acc.y);
-      mh = m_new;
-      fence_proxy_async_smem();  // P stores -> visible to the tensor core
+      // hand the row's sum, and the max it is relative to, to the epilogue
+      lfin[x * 128 + row] = l;
+      mfin[x * 128 + row] = m_run;
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_pfull(j % PB));
+      if (lane == 0) mbar_arrive(bar_epi(x));
     }
-    // hand the row's partial sum, and the max it is relative to, to the epilogue
-    lfin[h * 128 + row] = l;
-    mfin[h * 128 + row] = mh;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar_epi);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCorrectionRegs));
-    // ============================================================ two-level accumulation
+    // ============================================================ running-output rescale
+    // O_x = alpha O_x in FP32 before PV_x(j) adds the tile's P V block onto it; skipped
+    // by a warp whose 32 rows all keep their max (alpha = 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int grow = qt * kBlkQ + row;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tPV0 = tmem + lane_base + kColPV;
-    const uint32_t tO = tmem + lane_base + kColO;
     bool ok = !dead;
 
     for (int j = 0; j < nkv && ok; ++j) {
-      const int sa = j % kAlphaRing;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_afull(sa), (j / kAlphaRing) & 1, 0x401)) &&
-           __all_sync(0xffffffffu, mbar_wait(bar_pvfull(j & 1), (j >> 1) & 1, 0x402));
-      if (!ok) break;
-      tc_fence_after();
-      const float al = alph[sa * 128 + row];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_afree(sa));
-      const f2 AL = make_float2(al, al);
-      const uint32_t tPV = tPV0 + 128u * (j & 1);
-      // O = alpha * O + PV_blk, 32 columns at a time (the first tile just copies PV_blk)
+      for (int x = 0; x < nX && ok; ++x) {
+        const int sa = j % kAlphaRing;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_afull(x, sa), (j / kAlphaRing) & 1, 0x401 + x));
+        if (!ok) break;
+        const float al = alph[(x * kAlphaRing + sa) * 128 + row];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_afree(x, sa));
+        if (j == 0) continue;  // PV_x(0) starts O_x afresh
+        // O_x holds PV_x(j - 1) complete before it is rescaled
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_pvdone(x), (j - 1) & 1, 0x403 + x));
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, al != 1.0f)) {
+          const uint32_t tO = tmem + lane_base + kColO + 128u * x;
+          const f2 AL = make_float2(al, al);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t rp[32], ro[32];
-        tmem_ld32(tPV + 32u * c, rp);
-        if (j > 0) {
-          tmem_ld32(tO + 32u * c, ro);
-          tmem_wait_ld_tied(rp);
-          pin_regs(ro);
-        } else {
-          tmem_wait_ld_tied(rp);
-        }
-        if (c == D / 32 - 1) {  // the whole PV block has been read: PV(j + 2) may run
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_pvfree(j & 1));
-        }
-        if (j > 0) {
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ro[32];
+            tmem_ld32(tO + 32u * c, ro);
+            tmem_wait_ld_tied(ro);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const f2 o = f2_fma(pair_of(ro, i), AL, pair_of(rp, i));
-            ro[2 * i] = __float_as_uint(o.x);
-            ro[2 * i + 1] = __float_as_uint(o.y);
+            for (int i = 0; i < 16; ++i) {
+              const f2 o = f2_mul(pair_of(ro, i), AL);
+              ro[2 * i] = __float_as_uint(o.x);
+              ro[2 * i + 1] = __float_as_uint(o.y);
+            }
+            tmem_st32(tO + 32u * c, ro);
           }
-          tmem_st32(tO + 32u * c, ro);
-        } else {
-          tmem_st32(tO + 32u * c, rp);
+          tmem_wait_st();
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_oready(x));
       }
-      tmem_wait_st();
     }
 
     // ---------------------------------------------------------------- epilogue
-    ok = ok && __all_sync(0xffffffffu, mbar_wait<true>(bar_epi, 0, 0x403));
-    if (ok) {
+    const float* vs = a.v_scale + (static_cast<int64_t>(b) * a.hkv + hk) * D;
+    for (int x = 0; x < nX && ok; ++x) {
+      ok = __all_sync(0xffffffffu, mbar_wait<true>(bar_pvdone(x), (nkv - 1) & 1, 0x405 + x)) &&
+           __all_sync(0xffffffffu, mbar_wait<true>(bar_epi(x), 0, 0x407 + x));
+      if (!ok) break;
       tc_fence_after();
-      // the two warpgroups' sums are relative to the max of their own last tile;
-      // the overall max is that of the last tile
-      const double m0 = mfin[row], m1 = mfin[128 + row];
-      const double m = fmax(m0, m1);
-      const float l = lfin[row] * ex2(static_cast<float>((m0 - m) * kLog2E64)) +
-                      lfin[128 + row] * ex2(static_cast<float>((m1 - m) * kLog2E64));
+      const int grow = (2 * qp + x) * kBlkQ + row;
+      const double m = mfin[x * 128 + row];
+      const float l = lfin[x * 128 + row];
       const float inv_l = 1.0f / l;
-      const float* vs = a.v_scale + (static_cast<int64_t>(b) * a.hkv + hk) * D;
+      const uint32_t tO = tmem + lane_base + kColO + 128u * x;
       const int64_t orow =
           seq_base(seq, b, a.osb, a.ost) + hq * a.osh + static_cast<int64_t>(grow) * a.ost;
 #pragma unroll

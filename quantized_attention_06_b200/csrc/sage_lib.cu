@@ -76,9 +76,10 @@ sage_status_t plan(const sage_problem_t* p, Layout& L, SeqVarlen* storage) {
         storage->cta[b] = static_cast<int32_t>(cta);
         if (b < p->batch) {
           const int n = cu[b + 1] - cu[b];
-          const int tiles = (n + kBlkQ - 1) / kBlkQ;  // one attention CTA per 128-row Q tile
+          // one attention CTA per pair of 128-row Q tiles
+          const int pairs = ((n + kBlkQ - 1) / kBlkQ + 1) / 2;
           off += static_cast<int64_t>(round_up(n, kPad));
-          cta += static_cast<int64_t>(p->heads_q) * tiles;
+          cta += static_cast<int64_t>(p->heads_q) * pairs;
         }
       }
       L.var = storage;
@@ -500,8 +501,8 @@ sage_status_t sage_attn_fwd(const sage_problem_t* p, const int8_t* q8, const flo
     if (ncta == 0) return SAGE_OK;
     return dispatch_attn(*L.var, ncta, d, fine, pv, mq, mk, mv, a, s);
   }
-  const int64_t tiles = (L.dense.len + kBlkQ - 1) / kBlkQ;
-  const int64_t ncta = static_cast<int64_t>(p->batch) * p->heads_q * tiles;
+  const int64_t pairs = ((L.dense.len + kBlkQ - 1) / kBlkQ + 1) / 2;
+  const int64_t ncta = static_cast<int64_t>(p->batch) * p->heads_q * pairs;
   return dispatch_attn(L.dense, ncta, d, fine, pv, mq, mk, mv, a, s);
 }
 
