@@ -220,12 +220,16 @@ sage_status_t sage_quant_qkv(const sage_problem_t* p,
  *          scales of row i's Q block and key j's K block at the problem's granularity)
  *   causal: x_j = -inf for j > i
  *   m'   = max(m, max_j x_j);   P~_j = exp(x_j - m');   l = l e^{m-m'} + sum_j P~_j
- *   P8   = e4m3(448 P~);  PV_blk = P8 V8 (FP32, fresh per block);  O = O e^{m-m'} + PV_blk
+ *   P8   = e4m3(448 P~);  O = O e^{m-m'} + PV_blk,  PV_blk = P8 V8
  *   out  = O * v_scale / (448 l)           lse = m + ln(l)   (natural log)
  *   (SAGE_PV_FP16: P = P~ rounded to the input's 16-bit type, PV_blk = P V16,
  *    out = O / l.)
- * The logits, the running max and the exponent argument are formed in fp32 and
- * exp is the hardware base-2 exponential (within 2 ulp of exact).
+ * The logits x and the running max m are fp64.  O is an FP32 accumulator in TMEM:
+ * each block it is rescaled by e^{m-m'} in FP32 and the tensor core adds the block's
+ * P8 V8 onto it in FP32.  P~ is formed in fp32 with the hardware base-2 exponential
+ * from fp64-formed constants; every e4m3 code whose fp32 P~ lies within 32 ulps of a
+ * rounding midpoint is decided again in fp64, so the codes are those of the fp64
+ * definition.
  * sm_scale <= 0 selects 1/sqrt(head_dim).  is_causal != 0 applies the mask above.
  * out: written in out_dtype (SAGE_FP16, SAGE_BF16 or SAGE_FP32) with element
  * strides out_strides {batch, head, token}, last dimension contiguous, the
