@@ -91,6 +91,7 @@ struct AttnCfg {
   static constexpr int kKS = PV == kPvE4m3 ? 3 : 2;      // K ring stages
   static constexpr int kVS = PV == kPvE4m3 ? 3 : 2;      // V ring stages
   static constexpr int kPBufs = PV == kPvE4m3 ? 2 : 1;   // P tiles in shared memory per Q tile
+  static_assert(kPBufs == 1 || kPBufs == 2, "the barrier-free buffer reuse assumes two P buffers");
   static constexpr int kTileQK = kBlkQ * D;              // bytes of one Q (or K) tile
   static constexpr int kTileV = D * kKvTile * kEB;       // bytes of one V^T tile
   static constexpr int kTileP = kBlkQ * kKvTile * kEB;   // bytes of one P tile
@@ -727,7 +728,12 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const double m_new = fmax(m_run, mt);
         // alpha = e^(m - m') rescales l here and O in the correction warps (slot j % 4)
         const float alpha = ex2(static_cast<float>((m_run - m_new) * kLog2E64));
-        if (j >= kAlphaRing) {
+        // With two P buffers no wait is needed before reusing alpha slot j % 4 or P buffer
+        // j % 2: the commit that completed S(j) covers every earlier MMA of this Q tile's
+        // issuer, PV(j - 2) among them, and PV(j - 2) was issued only after the correction
+        // warps had read alpha(j - 2) (they read the alphas in tile order).  With one P
+        // buffer (16-bit P) PV(j - 1) is issued after S(j), so both waits stay.
+        if (PB == 1 && j >= kAlphaRing) {
           const int jo = j - kAlphaRing;
           ok = __all_sync(0xffffffffu, mbar_wait(bar_afree(x, jo % kAlphaRing), (jo / kAlphaRing) & 1, 0x305 + x));
           if (!ok) break;
@@ -735,27 +741,38 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         alph[(x * kAlphaRing + j % kAlphaRing) * 128 + row] = alpha;
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_afull(x, j % kAlphaRing));
+        // per K-scale block: c = q_scale k_scale sm_scale log2 e and
+        // nb = S_max c - m' log2 e + log2 ps, in fp64, each rounded once (formed while the
+        // P buffer may still be in use where registers allow: with e4m3 P)
+        float ckb[kSB], nbb[kSB];
+        if constexpr (PV == kPvE4m3) {
+          const double ml = __dmul_rn(m_new, kLog2E64);
+#pragma unroll
+          for (int bb = 0; bb < kSB; ++bb) {
+            const double cc = chunk_cc(sq_sc, skd[bb]);
+            ckb[bb] = chunk_ck(cc);
+            nbb[bb] = chunk_nb(hb[bb], cc, ml, kLog2Ps);
+          }
+        }
         // the P buffer of tile j was last read by PV(j - PB)
         const int pb = j % PB;
-        if (j >= PB) {
+        if (PB == 1 && j >= PB) {
           const int jo = j - PB;
           ok = __all_sync(0xffffffffu, mbar_wait(bar_pfree(x, jo % PB), (jo / PB) & 1, 0x307 + x));
           if (!ok) break;
         }
-
-        // per K-scale block: c = q_scale k_scale sm_scale log2 e and
-        // nb = S_max c - m' log2 e + log2 ps, in fp64, each rounded once
-        const double ml = __dmul_rn(m_new, kLog2E64);
+        if constexpr (PV != kPvE4m3) {
+          const double ml = __dmul_rn(m_new, kLog2E64);
+#pragma unroll
+          for (int bb = 0; bb < kSB; ++bb) {
+            const double cc = chunk_cc(sq_sc, skd[bb]);
+            ckb[bb] = chunk_ck(cc);
+            nbb[bb] = chunk_nb(hb[bb], cc, ml, kLog2Ps);
+          }
+        }
         const uint32_t ptile = sbase + L::kPOff + (x * PB + pb) * L::kTileP;
         const uint32_t prow = ptile + row * 128;
         f2 acc = make_float2(0.0f, 0.0f);
-        float ckb[kSB], nbb[kSB];
-#pragma unroll
-        for (int bb = 0; bb < kSB; ++bb) {
-          const double cc = chunk_cc(sq_sc, skd[bb]);
-          ckb[bb] = chunk_ck(cc);
-          nbb[bb] = chunk_nb(hb[bb], cc, ml, kLog2Ps);
-        }
         uint32_t flag = 0u;  // lane c < 4: which rows of this warp have a flagged p in chunk c
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -821,7 +838,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         if (!ok) break;
         const float al = alph[(x * kAlphaRing + sa) * 128 + row];
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_afree(x, sa));
+        if (PB == 1 && lane == 0) mbar_arrive(bar_afree(x, sa));
         if (j == 0) continue;  // PV_x(0) starts O_x afresh
         // O_x holds PV_x(j - 1) complete before it is rescaled
         ok = __all_sync(0xffffffffu, mbar_wait(bar_pvdone(x), (j - 1) & 1, 0x403 + x));
