@@ -151,17 +151,15 @@ quant_fused_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const SeqPos sp = locate(seq, pb * kPad, 0, 0);
     const int row = (std::is_same<Seq, SeqVarlen>::value ? seq_base(seq, sp.b, 0, 1) : 0) +
                     (pb * kPad - sp.off);
-    int co[4] = {0, 0, 0, 0};
-    co[a.dim_tok] = row;
-    co[a.dim_head] = h;
-    co[a.dim_batch] = std::is_same<Seq, SeqVarlen>::value ? 0 : sp.b;
+    const int bco = std::is_same<Seq, SeqVarlen>::value ? 0 : sp.b;
+    auto coord = [&](int d) { return a.dim_tok == d ? row : a.dim_head == d ? h : a.dim_batch == d ? bco : 0; };
     const CUtensorMap* m = tensor == 0 ? &tmap_q : tensor == 1 ? &tmap_k : &tmap_v;
     const uint32_t st = slot % kFusedStages;
     const uint32_t dst = sbase + st * L::kTile;
     mbar_arrive_expect_tx(bar0 + 8u * st, L::kTile);
 #pragma unroll
     for (int bx = 0; bx < D / 64; ++bx)
-      tma_load_4d(dst + bx * L::kBox, m, 64 * bx, co[1], co[2], co[3], bar0 + 8u * st);
+      tma_load_4d(dst + bx * L::kBox, m, 64 * bx, coord(1), coord(2), coord(3), bar0 + 8u * st);
   };
 
   // ------------------------------------------------------------ per-unit work
@@ -260,10 +258,13 @@ quant_fused_kernel(const __grid_constant__ CUtensorMap tmap_q,
           float m = 0.0f;
 #pragma unroll
           for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[p][i]));
-          bm[isq ? 0 : (p / KB)] = fmaxf(bm[isq ? 0 : (p / KB)], m);
+          bm[p / KB] = fmaxf(bm[p / KB], m);  // K: each 64-row block; Q merges them below
         }
+        if (isq) bm[0] = fmaxf(bm[0], bm[1]);
         const int nb = isq ? 1 : 2;
-        for (int k2 = 0; k2 < nb; ++k2) {
+#pragma unroll
+        for (int k2 = 0; k2 < 2; ++k2) {
+          if (k2 >= nb) break;  // uniform over the CTA (the unit's tensor)
           const float amax = cta_max(bm[k2], redf);
           const float r = (amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
 #pragma unroll
@@ -298,9 +299,13 @@ quant_fused_kernel(const __grid_constant__ CUtensorMap tmap_q,
           float m = 0.0f;
 #pragma unroll
           for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[p][i]));
-          // rows of pass p lie in 32-row blocks (p*RPP + rr) / 32
-          bm[(p * RPP + rr) / F] = fmaxf(bm[(p * RPP + rr) / F], m);
+          // rows of pass p lie in 32-row block (p*RPP + rr) / 32 (a select per block keeps
+          // the array in registers)
+          const int blk = (p * RPP + rr) / F;
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) bm[k4] = blk == k4 ? fmaxf(bm[k4], m) : bm[k4];
         }
+#pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           const float amax = cta_max(bm[k4], redf);
           const float r = (amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
@@ -330,16 +335,19 @@ quant_fused_kernel(const __grid_constant__ CUtensorMap tmap_q,
     // chunk and 32 token groups, so each channel row leaves as 128 (or 256) contiguous bytes.
     const int cv = tid >> 5, tg = tid & 31;  // 16 chunks x 32 groups (d = 128)
     if (cv < CPR) {
+      // slot k holds token (k + tg) % 4 of the thread's four (read in that rotated order so
+      // a warp's reads spread over the banks); the packed codes are rotated back to token
+      // order with one funnel shift, so every index here is a compile-time one
+      const int rot = tg & 3;
       float y[4][8];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const int kk = (k + tg) & 3;  // rotated so a warp's reads spread over the banks
-        const int r = 4 * tg + kk;
+        const int r = 4 * tg + ((k + rot) & 3);
         const uint4 v = lds16(tile + tile_off<D>(r, cv));
         float f[8];
         unpack8<T>(v, f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) y[kk][i] = (r < nvalid) ? f[i] : 0.0f;
+        for (int i = 0; i < 8; ++i) y[k][i] = (r < nvalid) ? f[i] : 0.0f;
       }
       const int64_t row0 = static_cast<int64_t>(h) * D + cv * 8;
       if (!a.pv16) {
@@ -350,17 +358,22 @@ quant_fused_kernel(const __grid_constant__ CUtensorMap tmap_q,
           const float r = (vm[i] > 0.0f) ? __fdiv_rn(448.0f, vm[i]) : 0.0f;
           const uint32_t lo = e4m3x2(__fmul_rn(y[0][i], r), __fmul_rn(y[1][i], r));
           const uint32_t hi = e4m3x2(__fmul_rn(y[2][i], r), __fmul_rn(y[3][i], r));
-          *reinterpret_cast<uint32_t*>(dst + static_cast<int64_t>(i) * seq.t_pad) = lo | (hi << 16);
+          const uint32_t w = lo | (hi << 16);  // byte k = slot k
+          *reinterpret_cast<uint32_t*>(dst + static_cast<int64_t>(i) * seq.t_pad) =
+              __funnelshift_l(w, w, 8 * rot);  // byte (k + rot) % 4 = slot k
         }
       } else {
         T* dst = reinterpret_cast<T*>(a.v8) + row0 * seq.t_pad + pb * kPad + 4 * tg;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          __align__(8) T w[4];
+          uint64_t w = 0;  // 16-bit value k = slot k
 #pragma unroll
-          for (int k = 0; k < 4; ++k) w[k] = from_f32<T>(y[k][i]);
-          *reinterpret_cast<uint2*>(dst + static_cast<int64_t>(i) * seq.t_pad) =
-              *reinterpret_cast<const uint2*>(w);
+          for (int k = 0; k < 4; ++k) {
+            const T t = from_f32<T>(y[k][i]);
+            w |= static_cast<uint64_t>(*reinterpret_cast<const uint16_t*>(&t)) << (16 * k);
+          }
+          if (rot != 0) w = (w << (16 * rot)) | (w >> (64 - 16 * rot));  // value (k + rot) % 4 = slot k
+          *reinterpret_cast<uint64_t*>(dst + static_cast<int64_t>(i) * seq.t_pad) = w;
         }
       }
     }
