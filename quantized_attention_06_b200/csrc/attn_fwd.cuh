@@ -7,24 +7,21 @@
 // variable lengths); glossary page "SageAttention(セージアテンション)" (FlashAttention-
 // compatible online softmax).
 //
-// CTA = one (sequence, query head, 128-row Q tile).  16 warps in four warpgroups,
-// registers traded with setmaxnreg (128 x 56 + 128 x 88 + 256 x 184 = 512 x 128,
-// the launch allocation):
-//   WG0  warp 0: TMA producer (Q once, K / V tiles into rings)
-//        warp 1: TMEM owner and S issuer, warp 2: PV issuer (one thread each); warp 3 idle
-//          S(j)  = Q8 K8(j)^T   tcgen05.mma kind::i8 -> the TMEM S buffer
-//          PV(j) = P(j) V(j)    tcgen05.mma kind::f8f6f4 (e4m3) or kind::f16, A = P from
-//                               shared memory -> PV block j % 2, a fresh FP32 accumulator
-//   WG1  softmax of the even KV tiles, WG2 of the odd ones (one thread per query row,
-//        a whole 128-key row each); consecutive tiles pass the running max through
-//        shared memory, so the two warpgroups work on different tiles at once
-//   WG3  two-level accumulation O = alpha O + PV(j) held in TMEM, and the epilogue
+// CTA = one (sequence, query head, pair of 128-row Q tiles A = 2 qp and B = 2 qp + 1).
+// 16 warps in four warpgroups, registers traded with setmaxnreg (128 x 56 + 128 x 88 +
+// 256 x 184 = 512 x 128, the launch allocation):
+//   WG0  warp 0: TMA producer (both Q tiles once, K / V tiles into rings shared by A and B)
+//        warps 1 and 2: the MMA issuers of Q tiles A and B (one thread each); warp 3 idle
+//          S_x(j)  = Q8_x K8(j)^T  tcgen05.mma kind::i8 -> the TMEM S buffer of tile x
+//          PV_x(j) = P_x(j) V(j)   tcgen05.mma kind::f8f6f4 (e4m3) or kind::f16, A = P from
+//                                  shared memory, accumulated onto O_x in FP32
+//   WG1  softmax of Q tile A, WG2 of Q tile B (one thread per query row, a whole 128-key
+//        row each; the running max and sum stay in the thread's registers)
+//   WG3  the running-output rescale O_x = alpha O_x before PV_x(j), and the epilogue
 //
-// TMEM columns: the S buffer [0,128), PV blocks 0 and 1 at [128, 128 + d) and
-// [256, 256 + d), the running O at [384, 384 + d).  A softmax warpgroup loads S(j) into
-// registers and frees the buffer at once (P goes to shared memory), so S(j + 1) is
-// computed while P(j) is being formed.  PV(j) lands in block j % 2 and the correction
-// warps fold it into O while PV(j + 1) runs in the other block.
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256 + d), O_B [384, 384 + d).  A
+// softmax warpgroup loads S_x(j) into registers and frees the buffer at once (P goes to
+// shared memory), so S_x(j + 1) is computed while P_x(j) is being formed.
 // Every S accumulates onto the magic pattern 0x4B400000 (fp32 1.5 * 2^23), so TMEM
 // returns bits(12582912 + S).  The pattern is written by the tensor core itself: before
 // the INT8 steps of S(j), one kind::f16 MMA with constant operands (every A entry 512,
@@ -35,9 +32,9 @@
 //   m'    = max(m, max_j x_ij)                      (fp64, as the definition)
 //   p_j   = ps exp(x_j - m')                        (ps = 448 for e4m3 P, 1 for 16-bit P)
 //   l     = l exp(m - m') + sum_j p_j   (unquantized),  P_j = round(p_j) -> smem
-//   O     = O exp(m - m') + PV_blk      (PV_blk = P V in FP32, fresh each tile)
+//   O     = O exp(m - m') + P V         (FP32 in TMEM: rescaled, then the tile's block added)
 //   out   = O v_scale / l ;  lse = m' + ln(l / ps)
-// p is computed in the log2 domain from fp32 operations relative to each 32-key chunk's
+// p is computed in the log2 domain from fp32 operations relative to each K-scale block's
 // own largest score, t = fma(S - S_max_c, c_c, nb_c) with c_c = q_scale k_scale_c sm_scale
 // log2 e and nb_c = S_max_c c_c - m' log2 e + log2 ps formed in fp64 and rounded once,
 // and 2^t is the hardware exponential (ex2.approx, within 2 ulp).  That p is within
